@@ -1,0 +1,184 @@
+/*
+ * idx.h — C ABI of libidx.so, a B200 (sm_100a) implementation of the
+ * DeepSeek-V3.2 lightning indexer's hot path:
+ *
+ *   keys:    rotate (scaled Hadamard-128) → block-FP8 quantise → append to the
+ *            per-sequence FP8 key cache;
+ *   scores:  S[t,s] = k_scale[s] · Σ_{h<64} w[t,h] · ReLU(q_fp8[t,h] · k_fp8[s]);
+ *   select:  the min(k, visible) highest-scoring cached positions per query row.
+ *
+ * Sources (web pages on DeepSeek-V3.2-Exp's lightning indexer):
+ *   "Index scores"          — score equation S^I, fp8_index docstring, Indexer.forward excerpt;
+ *   "Index key cache"       — k_cache / k_scale_cache buffers, append before scoring;
+ *   "Hadamard rotation"     — rotation equation and orthonormality note;
+ *   NKI "DeepSeek-V3.2 Sparse Indexer Kernel API Reference" — caller-owned cache written in
+ *                             place, int32 positions, int32 unordered top-k set.
+ *
+ * Conventions for every call below.
+ *   - All array arguments are DEVICE pointers to row-major, contiguous memory
+ *     owned by the caller.  The library never allocates device memory and never
+ *     synchronises in these calls; work is enqueued on `stream` (a cudaStream_t;
+ *     NULL = the legacy default stream) and runs asynchronously.
+ *   - bf16 arrays are passed as uint16_t bit patterns; FP8 arrays hold e4m3fn
+ *     codes as uint8_t.
+ *   - Index head count H = 64 and head dimension D = 128 are fixed.
+ *   - Return value: IDX_OK (0) when the work was enqueued, or a negative IDX_ERR_*
+ *     for an argument error detected on the host (nothing is enqueued then).
+ *     Errors that depend on device data (positions, lengths) are detected in the
+ *     kernels, which then skip the offending sequence and set a bit in a device
+ *     error word; idx_status() reports and clears it.
+ *   - Query row i (0 ≤ i < n) of sequence b sits at position lengths[b] − n + i
+ *     (the call's new rows are the last n cached positions).  Key s is visible to
+ *     that row iff s < lengths[b] and, when causal != 0, s ≤ its position.
+ *     visible(b,i) = causal ? lengths[b] − n + i + 1 : lengths[b].
+ *   - Scale format `fmt`: IDX_FMT_FP32 stores scale = fl32(max(amax,1e-4)/448);
+ *     IDX_FMT_UE8M0 rounds that up to a power of two.  Both store float32.
+ */
+#ifndef IDX_H_
+#define IDX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define IDX_API __attribute__((visibility("default")))
+#else
+#define IDX_API
+#endif
+
+typedef struct CUstream_st* idx_stream_t;
+
+#define IDX_HEADS 64
+#define IDX_DIM 128
+#define IDX_MAX_LEN 131072 /* largest lengths[b] / max_len a score call accepts */
+
+enum idx_fmt { IDX_FMT_FP32 = 0, IDX_FMT_UE8M0 = 1 };
+
+enum idx_status_code {
+  IDX_OK = 0,
+  IDX_ERR_NULL = -1,        /* a required pointer is NULL */
+  IDX_ERR_SHAPE = -2,       /* a size is negative, zero where it must not be, or too large */
+  IDX_ERR_FMT = -3,         /* fmt is not IDX_FMT_FP32 / IDX_FMT_UE8M0 */
+  IDX_ERR_K = -4,           /* k <= 0 */
+  IDX_ERR_ALIGN = -5,       /* a pointer is not 16-byte aligned where required */
+  IDX_ERR_LAUNCH = -6,      /* the CUDA launch failed (the CUDA error is in idx_last_cuda_error) */
+  IDX_ERR_DEVICE = -7,      /* idx_status: a kernel set the device error word */
+  IDX_ERR_CUDA = -8,        /* idx_status: the stream itself reported a CUDA error */
+  IDX_ERR_UNSUPPORTED = -9  /* no device code for this GPU (not sm_100) */
+};
+
+/* Bits of the device error word (returned by idx_device_error_bits). */
+#define IDX_DEV_ERR_TIMEOUT 0x1u  /* a bounded wait inside a kernel gave up */
+#define IDX_DEV_ERR_POSITION 0x2u /* idx_quant_append: positions[b] < 0 or positions[b] + n > T_cap */
+#define IDX_DEV_ERR_LENGTH 0x4u   /* score/top-k: lengths[b] < n or lengths[b] > max_len */
+
+/*
+ * idx_quant — "Hadamard rotation" page (rotation equation) followed by the
+ * block-FP8 quantisation of groups of 128 features.
+ *   x_bf16  [rows, 128]  bf16 input rows.
+ *   x_fp8   [rows, 128]  out: e4m3 codes of fl32(y / scale), y = bf16(H·x/√128).
+ *   x_scale [rows]       out: float32 scale per row.
+ * rows may be 0 (nothing is enqueued).  x_bf16 and x_fp8 must be 8-byte aligned.
+ */
+IDX_API int idx_quant(const uint16_t* x_bf16, int64_t rows, uint8_t* x_fp8, float* x_scale, int fmt,
+              idx_stream_t stream);
+
+/*
+ * idx_quant_queries — queries of `tokens` rows of 64 heads: the same rotation
+ * and quantisation per (token, head), and the head weights folded as on the
+ * "Index scores" page (1/√64 into the weights, 1/√128 with the query's scale):
+ *   w[t,h] = fl32(fl32(fl32(w_raw[t,h]·0.125)·q_scale[t,h])·fl32(128^-1/2)).
+ *   q_bf16 [tokens, 64, 128], w_raw [tokens, 64] float32 in;
+ *   q_fp8 [tokens, 64, 128] out; w [tokens, 64] float32 out (the folded weights
+ *   idx_score / idx_score_topk take).  The query scales are not stored.
+ */
+IDX_API int idx_quant_queries(const uint16_t* q_bf16, const float* w_raw, int64_t tokens, uint8_t* q_fp8, float* w,
+                      int fmt, idx_stream_t stream);
+
+/*
+ * idx_quant_append — "Index key cache" page: rotate and quantise n new keys of
+ * each of B sequences and write them in place at slots positions[b] … +n−1.
+ *   k_bf16        [B, n, 128] bf16.
+ *   positions     [B] int32 first slot per sequence.
+ *   k_cache       [B, T_cap, 128] uint8 (e4m3), written in place.
+ *   k_scale_cache [B, T_cap] float32, written in place.
+ * A sequence with positions[b] < 0 or positions[b] + n > T_cap is skipped and
+ * IDX_DEV_ERR_POSITION is raised.
+ */
+IDX_API int idx_quant_append(const uint16_t* k_bf16, const int32_t* positions, int B, int n, uint8_t* k_cache,
+                     float* k_scale_cache, int T_cap, int fmt, idx_stream_t stream);
+
+/*
+ * idx_score — "Index scores" page: score equation and fp8_index docstring
+ * (FP8 q·k → fp32 logits, ReLU, × head weight, sum over heads, × key scale),
+ * with the causal mask of the Indexer.forward excerpt.
+ *   q_fp8  [B, n, 64, 128] e4m3 codes; w [B, n, 64] folded weights (idx_quant_queries).
+ *   k_cache [B, T_cap, 128], k_scale_cache [B, T_cap]; lengths [B] int32.
+ *   max_len: host-side upper bound on lengths[b] (n ≤ max_len ≤ min(T_cap, IDX_MAX_LEN));
+ *            it sizes the launch.
+ *   scores [B, n, ld] float32 out: S for visible keys, −inf for every other column < ld.
+ *          ld ≥ 1; columns ≥ ld are not computed.
+ * q_fp8 and k_cache must be 16-byte aligned (they are read by TMA).
+ */
+IDX_API int idx_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
+              const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, float* scores, int64_t ld,
+              idx_stream_t stream);
+
+/*
+ * idx_topk — Indexer.forward excerpt (top min(index_topk, ·) per row) and the
+ * NKI page's output convention (int32, unordered set), on scores already in memory.
+ *   scores [B, n, ld] float32 (finite for visible keys); lengths [B]; causal as above.
+ *   indices [B, n, k] int32 out: the k_t = min(k, visible(b,i)) positions with the
+ *   highest scores, in unspecified order, in columns 0 … k_t−1; columns k_t … k−1
+ *   hold −1.  Ties at the k_t-th score are broken arbitrarily.
+ *   max_len as in idx_score (and ≤ ld).  ws / ws_bytes: reserved, pass NULL / 0.
+ */
+IDX_API int idx_topk(const float* scores, const int32_t* lengths, int B, int n, int64_t ld, int max_len, int causal, int k,
+             int32_t* indices, void* ws, size_t ws_bytes, idx_stream_t stream);
+
+/*
+ * idx_score_topk — idx_score followed by idx_topk in one kernel: the scores of
+ * a row never leave on-chip memory.  Arguments as in idx_score / idx_topk.
+ */
+IDX_API int idx_score_topk(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
+                   const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, int k,
+                   int32_t* indices, void* ws, size_t ws_bytes, idx_stream_t stream);
+
+/* Scratch bytes idx_topk / idx_score_topk need for these sizes (currently 0). */
+IDX_API size_t idx_workspace_size(int B, int n, int T_cap, int k);
+
+/*
+ * idx_status — synchronises `stream`, then reads and clears the device error
+ * word.  Returns IDX_OK, IDX_ERR_DEVICE (bits available from
+ * idx_device_error_bits) or IDX_ERR_CUDA.
+ */
+IDX_API int idx_status(idx_stream_t stream);
+IDX_API unsigned int idx_device_error_bits(void); /* bits seen by the last idx_status call */
+IDX_API const char* idx_error_string(int code);
+IDX_API int idx_last_cuda_error(void); /* cudaError_t of the last failed launch, 0 if none */
+
+/*
+ * idx_e4m3_encode — the float32 → e4m3fn conversion the quantiser uses (round to
+ * nearest even, saturate to ±448, sign of zero kept), exposed so that it can be
+ * checked value by value.  x [count] float32 in, out [count] uint8 codes.
+ */
+IDX_API int idx_e4m3_encode(const float* x, int64_t count, uint8_t* out, idx_stream_t stream);
+
+/*
+ * Fault-injection control for tests: when `flags` has bit 0 set, the next score
+ * launches make one bounded wait in each CTA wait for a barrier that nothing
+ * signals, with the wait budget set to `budget_ns`; the kernels then report
+ * IDX_DEV_ERR_TIMEOUT and return.  idx_debug_set(0, 0) restores normal
+ * operation (2 s wait budget).
+ */
+IDX_API void idx_debug_set(unsigned int flags, unsigned long long budget_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IDX_H_ */

@@ -236,13 +236,14 @@ def visible_count(length: int, n: int, i: int, causal: bool) -> int:
 
 
 def index_scores(q_codes, w, k_cache, k_scale_cache, lengths, causal, ncols=None,
-                 with_bound=True):
+                 with_bound=True, rows=None, seqs=None):
     """S[b, i, s] = k_scale[s] · Σ_h w[b,i,h] · max(L, 0),  L = Σ_d q·k exact.
 
     q_codes [B, n, 64, 128] uint8; w [B, n, 64] float32; k_cache [B, T, 128]
     uint8; k_scale_cache [B, T] float32.  Returns float64 arrays S and E (the
     per-entry bound |k_scale| · Σ_h |w·L|) of shape [B, n, ncols]; masked
-    entries of S are −inf and of E are 0.
+    entries of S are −inf and of E are 0.  ``rows`` / ``seqs`` restrict the
+    computation to some query rows / sequences (the others stay −inf).
     """
     q_codes = np.asarray(q_codes, np.uint8)
     B, n = q_codes.shape[:2]
@@ -251,13 +252,13 @@ def index_scores(q_codes, w, k_cache, k_scale_cache, lengths, causal, ncols=None
         ncols = int(lengths.max()) if B else 0
     S = np.full((B, n, ncols), -np.inf)
     E = np.zeros((B, n, ncols))
-    for b in range(B):
+    for b in (range(B) if seqs is None else seqs):
         L_b = int(lengths[b])
         if L_b == 0:
             continue
         kd = e4m3_decode(k_cache[b, :L_b])                       # [L_b, 128]
         ks = np.asarray(k_scale_cache[b, :L_b], np.float64)
-        for i in range(n):
+        for i in (range(n) if rows is None else rows):
             v = min(visible_count(L_b, n, i, causal), ncols)
             if v <= 0:
                 continue

@@ -1,0 +1,184 @@
+"""ctypes binding of libidx.so: argument marshalling only.
+
+Every function here checks tensor placement, dtype and contiguity, passes raw
+device pointers and the current CUDA stream to the C ABI declared in
+include/idx.h, and raises on a non-zero status.  All arithmetic happens in the
+library's CUDA kernels; there is no fallback path: if libidx.so is missing or
+the device is not an sm_100 GPU, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libidx.so")
+
+FMT_FP32 = 0
+FMT_UE8M0 = 1
+HEADS = 64
+DIM = 128
+DEV_ERR_TIMEOUT = 0x1
+DEV_ERR_POSITION = 0x2
+DEV_ERR_LENGTH = 0x4
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+# name → (restype, argtypes); mirrors include/idx.h
+SIGNATURES = {
+    "idx_quant": (_I, [_P, _I64, _P, _P, _I, _P]),
+    "idx_quant_queries": (_I, [_P, _P, _I64, _P, _P, _I, _P]),
+    "idx_quant_append": (_I, [_P, _P, _I, _I, _P, _P, _I, _I, _P]),
+    "idx_score": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P]),
+    "idx_topk": (_I, [_P, _P, _I, _I, _I64, _I, _I, _I, _P, _P, _SZ, _P]),
+    "idx_score_topk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
+    "idx_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "idx_status": (_I, [_P]),
+    "idx_device_error_bits": (ctypes.c_uint, []),
+    "idx_error_string": (ctypes.c_char_p, [_I]),
+    "idx_last_cuda_error": (_I, []),
+    "idx_e4m3_encode": (_I, [_P, _I64, _P, _P]),
+    "idx_debug_set": (None, [ctypes.c_uint, ctypes.c_ulonglong]),
+}
+
+_lib = None
+
+
+class IdxError(RuntimeError):
+    pass
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libidx.so (once) and declare its signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise IdxError(f"{path} is missing: build it with `python -m sparse_attention_token_idx_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        lib = load()
+        msg = lib.idx_error_string(code).decode()
+        raise IdxError(f"{what}: {msg} (status {code}, cuda error {lib.idx_last_cuda_error()})")
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None, dtype=None, name="tensor") -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise IdxError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise IdxError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise IdxError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+_BF16 = (torch.bfloat16, torch.int16, torch.uint16)
+
+
+def quant(x: torch.Tensor, fmt: int, out=None, scale=None, stream=None):
+    """Rotate + quantise rows of 128 bf16 features → (e4m3 codes uint8, scale fp32)."""
+    rows = x.numel() // DIM
+    codes = out if out is not None else torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scale = scale if scale is not None else torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _check(load().idx_quant(_ptr(x, _BF16, "x"), rows, _ptr(codes, torch.uint8, "out"),
+                            _ptr(scale, torch.float32, "scale"), fmt, _stream(stream)), "idx_quant")
+    return codes, scale
+
+
+def quant_queries(q: torch.Tensor, w_raw: torch.Tensor, fmt: int, q_out=None, w_out=None, stream=None):
+    """Queries [..., 64, 128] bf16 + raw head weights [..., 64] → (q codes, folded weights)."""
+    tokens = q.numel() // (HEADS * DIM)
+    q_out = q_out if q_out is not None else torch.empty(q.shape, dtype=torch.uint8, device=q.device)
+    w_out = w_out if w_out is not None else torch.empty(w_raw.shape, dtype=torch.float32, device=q.device)
+    _check(load().idx_quant_queries(_ptr(q, _BF16, "q"), _ptr(w_raw, torch.float32, "w_raw"), tokens,
+                                    _ptr(q_out, torch.uint8, "q_out"), _ptr(w_out, torch.float32, "w_out"), fmt,
+                                    _stream(stream)), "idx_quant_queries")
+    return q_out, w_out
+
+
+def quant_append(k_new: torch.Tensor, positions: torch.Tensor, k_cache: torch.Tensor,
+                 k_scale_cache: torch.Tensor, fmt: int, stream=None):
+    """Rotate, quantise and write k_new [B, n, 128] at slots positions[b] … (in place)."""
+    B, n = k_new.shape[0], k_new.shape[1]
+    T_cap = k_cache.shape[1]
+    _check(load().idx_quant_append(_ptr(k_new, _BF16, "k_new"), _ptr(positions, torch.int32, "positions"), B, n,
+                                   _ptr(k_cache, torch.uint8, "k_cache"),
+                                   _ptr(k_scale_cache, torch.float32, "k_scale_cache"), T_cap, fmt,
+                                   _stream(stream)), "idx_quant_append")
+
+
+def score(q_fp8, w, k_cache, k_scale_cache, lengths, causal: bool, max_len: int, ld: int | None = None,
+          out=None, stream=None):
+    """Scores [B, n, ld] fp32 (−inf outside each row's visible keys)."""
+    B, n = q_fp8.shape[0], q_fp8.shape[1]
+    T_cap = k_cache.shape[1]
+    ld = ld if ld is not None else max_len
+    out = out if out is not None else torch.empty((B, n, ld), dtype=torch.float32, device=q_fp8.device)
+    _check(load().idx_score(_ptr(q_fp8, torch.uint8, "q_fp8"), _ptr(w, torch.float32, "w"),
+                            _ptr(k_cache, torch.uint8, "k_cache"), _ptr(k_scale_cache, torch.float32, "k_scale"),
+                            _ptr(lengths, torch.int32, "lengths"), B, n, T_cap, max_len, int(causal),
+                            _ptr(out, torch.float32, "scores"), ld, _stream(stream)), "idx_score")
+    return out
+
+
+def topk(scores, lengths, causal: bool, k: int, max_len: int, out=None, stream=None):
+    """Top-k positions [B, n, k] int32 (a set per row, −1 padded) of materialised scores [B, n, ld]."""
+    B, n, ld = scores.shape
+    out = out if out is not None else torch.empty((B, n, k), dtype=torch.int32, device=scores.device)
+    _check(load().idx_topk(_ptr(scores, torch.float32, "scores"), _ptr(lengths, torch.int32, "lengths"), B, n, ld,
+                           max_len, int(causal), k, _ptr(out, torch.int32, "indices"), None, 0, _stream(stream)),
+           "idx_topk")
+    return out
+
+
+def score_topk(q_fp8, w, k_cache, k_scale_cache, lengths, causal: bool, k: int, max_len: int, out=None,
+               stream=None):
+    """Fused scores + top-k: positions [B, n, k] int32 (a set per row, −1 padded)."""
+    B, n = q_fp8.shape[0], q_fp8.shape[1]
+    T_cap = k_cache.shape[1]
+    out = out if out is not None else torch.empty((B, n, k), dtype=torch.int32, device=q_fp8.device)
+    _check(load().idx_score_topk(_ptr(q_fp8, torch.uint8, "q_fp8"), _ptr(w, torch.float32, "w"),
+                                 _ptr(k_cache, torch.uint8, "k_cache"),
+                                 _ptr(k_scale_cache, torch.float32, "k_scale"),
+                                 _ptr(lengths, torch.int32, "lengths"), B, n, T_cap, max_len, int(causal), k,
+                                 _ptr(out, torch.int32, "indices"), None, 0, _stream(stream)), "idx_score_topk")
+    return out
+
+
+def e4m3_encode(x: torch.Tensor, stream=None) -> torch.Tensor:
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(load().idx_e4m3_encode(_ptr(x, torch.float32, "x"), x.numel(), _ptr(out, torch.uint8, "out"),
+                                  _stream(stream)), "idx_e4m3_encode")
+    return out
+
+
+def status(stream=None) -> tuple[int, int]:
+    """(status code, device error bits); synchronises the stream and clears the device error word."""
+    lib = load()
+    code = lib.idx_status(_stream(stream))
+    return code, int(lib.idx_device_error_bits())
+
+
+def debug_set(flags: int, budget_ns: int = 0):
+    load().idx_debug_set(flags, budget_ns)

@@ -1,0 +1,181 @@
+// Library-wide host code: device error word, status, error strings, tensor-map
+// creation through the driver entry point, and the fault-injection switch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+#include "api_internal.h"
+#include "ptx.cuh"
+
+namespace idx {
+
+namespace {
+constexpr int kMaxDevicesForWord = 64;
+int current_device_for_word() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return (d >= 0 && d < kMaxDevicesForWord) ? d : 0;
+}
+}  // namespace
+
+__device__ unsigned int g_error_word = 0;
+
+unsigned int* device_error_word() {
+  static std::atomic<unsigned int*> addr[kMaxDevicesForWord];
+  const int d = current_device_for_word();
+  unsigned int* a = addr[d].load();
+  if (!a) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_error_word) != cudaSuccess) return nullptr;
+    a = static_cast<unsigned int*>(ptr);
+    addr[d].store(a);
+  }
+  return a;
+}
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sms[kMaxDevices];
+std::atomic<int> g_smem_optin[kMaxDevices];
+std::atomic<int> g_last_cuda_error{0};
+std::atomic<unsigned int> g_last_device_bits{0};
+std::atomic<unsigned int> g_debug_flags{0};
+std::atomic<unsigned long long> g_debug_budget{0};
+constexpr unsigned long long kDefaultBudgetNs = 2000000000ull;  // 2 s
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return (d >= 0 && d < kMaxDevices) ? d : 0;
+}
+}  // namespace
+
+int num_sms() {
+  const int d = current_device();
+  int v = g_sms[d].load();
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || v <= 0) v = 148;
+    g_sms[d].store(v);
+  }
+  return v;
+}
+
+int max_dynamic_smem() {
+  const int d = current_device();
+  int v = g_smem_optin[d].load();
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, d) != cudaSuccess || v <= 0)
+      v = 227 * 1024;
+    g_smem_optin[d].store(v);
+  }
+  return v;
+}
+
+int smem_per_sm() {
+  static std::atomic<int> cache[kMaxDevices];
+  const int d = current_device();
+  int v = cache[d].load();
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, d) != cudaSuccess || v <= 0)
+      v = 228 * 1024;
+    cache[d].store(v);
+  }
+  return v;
+}
+
+int check_launch() {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return IDX_OK;
+  g_last_cuda_error.store(static_cast<int>(e));
+  return e == cudaErrorNoKernelImageForDevice || e == cudaErrorInvalidDeviceFunction ? IDX_ERR_UNSUPPORTED
+                                                                                       : IDX_ERR_LAUNCH;
+}
+
+bool make_tmap_u8_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                     uint32_t box_rows) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return false;
+  if (reinterpret_cast<uintptr_t>(base) & 15) return false;
+  const cuuint64_t dims[3] = {inner, mid, outer};
+  const cuuint64_t strides[2] = {inner, inner * mid};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(inner), box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+DebugState debug_state() {
+  DebugState s;
+  s.flags = g_debug_flags.load();
+  const unsigned long long b = g_debug_budget.load();
+  s.budget_ns = b ? b : kDefaultBudgetNs;
+  return s;
+}
+
+}  // namespace idx
+
+using namespace idx;
+
+extern "C" int idx_status(idx_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    g_last_cuda_error.store(static_cast<int>(cudaGetLastError()));
+    return IDX_ERR_CUDA;
+  }
+  unsigned int bits = 0;
+  const unsigned int zero = 0;
+  if (cudaMemcpyFromSymbol(&bits, g_error_word, sizeof(bits)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) {
+    g_last_cuda_error.store(static_cast<int>(cudaGetLastError()));
+    return IDX_ERR_CUDA;
+  }
+  g_last_device_bits.store(bits);
+  return bits ? IDX_ERR_DEVICE : IDX_OK;
+}
+
+extern "C" unsigned int idx_device_error_bits(void) { return g_last_device_bits.load(); }
+
+extern "C" int idx_last_cuda_error(void) { return g_last_cuda_error.load(); }
+
+extern "C" const char* idx_error_string(int code) {
+  switch (code) {
+    case IDX_OK: return "ok";
+    case IDX_ERR_NULL: return "a required pointer is NULL";
+    case IDX_ERR_SHAPE: return "a size argument is out of range";
+    case IDX_ERR_FMT: return "fmt must be IDX_FMT_FP32 or IDX_FMT_UE8M0";
+    case IDX_ERR_K: return "k must be positive";
+    case IDX_ERR_ALIGN: return "a pointer is not aligned as required";
+    case IDX_ERR_LAUNCH: return "the CUDA launch failed";
+    case IDX_ERR_DEVICE: return "a kernel reported an error (see idx_device_error_bits)";
+    case IDX_ERR_CUDA: return "the stream reported a CUDA error";
+    case IDX_ERR_UNSUPPORTED: return "no device code for this GPU (sm_100a required)";
+    default: return "unknown status";
+  }
+}
+
+extern "C" size_t idx_workspace_size(int B, int n, int T_cap, int k) {
+  (void)B;
+  (void)n;
+  (void)T_cap;
+  (void)k;
+  return 0;
+}
+
+extern "C" void idx_debug_set(unsigned int flags, unsigned long long budget_ns) {
+  g_debug_flags.store(flags);
+  g_debug_budget.store(budget_ns);
+}

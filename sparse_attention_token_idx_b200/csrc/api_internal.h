@@ -1,0 +1,29 @@
+// Host-side helpers shared by the library's translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "../../include/idx.h"
+
+namespace idx {
+
+int num_sms();                       // SM count of the current device (cached per device)
+int check_launch();                  // IDX_OK, or IDX_ERR_LAUNCH after recording cudaGetLastError()
+int max_dynamic_smem();              // opt-in shared memory per block of the current device
+int smem_per_sm();                   // shared memory per SM of the current device
+
+// Tensor map for a [outer, mid, inner] uint8 array (row pitch `inner` bytes,
+// plane pitch mid·inner bytes), box {128 bytes, box_rows, 1}, 128-byte swizzle.
+bool make_tmap_u8_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                     uint32_t box_rows);
+
+unsigned int* device_error_word();  // device address of the error word on the current device
+
+struct DebugState {
+  unsigned int flags;
+  unsigned long long budget_ns;
+};
+DebugState debug_state();
+
+}  // namespace idx

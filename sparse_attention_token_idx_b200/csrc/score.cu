@@ -1,0 +1,464 @@
+// Index scores and fused top-k ("Index scores" page: score equation S^I and
+// the fp8_index docstring; causal mask and top-k from the Indexer.forward
+// excerpt).
+//
+// Work item = (sequence b, block of NT query rows), served by a cluster of G
+// CTAs that split the visible keys into contiguous slices.  Per CTA:
+//   warp 0      TMA producer: the NT·64 query heads once, then 128-key tiles of
+//               the FP8 cache (16 KB each, 128-byte swizzle) into a STAGES ring;
+//   warp 1      owns TMEM and issues tcgen05.mma kind::f8f6f4 with the keys on
+//               M (128 lanes) and the query heads on N (NT·64 columns), K = 128
+//               as four K = 32 steps, fp32 accumulators in NUM_ACC TMEM buffers;
+//   warps 2 …   epilogue: thread ↔ key (TMEM lane), reads its NT·64 logits,
+//               S = k_scale · Σ_h w_h · max(L_h, 0) in fp32 registers, masks
+//               keys past each row's visible count, and writes the score either
+//               to global memory (idx_score) or, as an order-preserving key,
+//               to shared memory for the cluster-wide select (idx_score_topk).
+// Every wait is bounded (2 s by default); a CTA that gives up raises
+// IDX_DEV_ERR_TIMEOUT, drains its outstanding copies and MMAs, frees TMEM and
+// returns, and the cluster agrees on skipping the select so that no CTA is
+// left at a cluster barrier.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "api_internal.h"
+#include "ptx.cuh"
+#include "select.cuh"
+
+namespace idx {
+
+namespace {
+
+constexpr int kTileKeys = 128;
+constexpr int kTileBytes = kTileKeys * IDX_DIM;  // 16 KB
+
+struct ScoreParams {
+  const float* w;            // [B, n, 64]
+  const float* k_scale;      // [B, T_cap]
+  const int32_t* lengths;    // [B]
+  float* scores;             // [B, n, ld] (unfused)
+  int32_t* indices;          // [B, n, k] (fused)
+  int64_t ld;
+  int B, n, T_cap, max_len, causal, k;
+  int G;                     // cluster size
+  int ntb;                   // query-row blocks per sequence
+  int chunk_cap;             // keys per CTA the shared score buffer holds
+  unsigned int debug_flags;
+  unsigned long long budget_ns;
+  unsigned int* err;         // device error word
+};
+
+template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS>
+struct Cfg {
+  static constexpr int N = NT * IDX_HEADS;
+  static constexpr int kThreads = (2 + EPI_WARPS) * 32;
+  static constexpr int kAccCols = NUM_ACC * N;
+  static constexpr int kTmemCols = kAccCols <= 32 ? 32 : kAccCols <= 64 ? 64 : kAccCols <= 128 ? 128
+                                 : kAccCols <= 256 ? 256 : 512;
+  static_assert(kAccCols <= 512, "TMEM holds 512 columns");
+  static_assert(EPI_WARPS % 4 == 0 && NT % (EPI_WARPS / 4) == 0, "epilogue split");
+  static constexpr int kTokPerWarp = NT / (EPI_WARPS / 4);
+  static constexpr int kQBytes = N * IDX_DIM;
+  // shared memory carve (offsets from a 1024-aligned base)
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffW = kOffK + STAGES * kTileBytes;
+  static constexpr int kOffBar = kOffW + N * 4;
+  static constexpr int kNumBars = 2 * STAGES + 2 * NUM_ACC + 3;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kOffSel = (kOffMisc + 64 + 127) / 128 * 128;
+  static constexpr int kOffScores = kOffSel + (FUSED ? static_cast<int>(sizeof(SelectSmem)) : 0);
+  static int smem_bytes(int chunk_cap) {
+    return 1024 + kOffScores + (FUSED ? NT * chunk_cap * 4 : 0);
+  }
+};
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS>
+__global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>::kThreads, 1)
+    score_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
+                 const ScoreParams p) {
+  using C = Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>;
+  constexpr int N = C::N;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_s = smem + C::kOffQ;
+  uint8_t* k_s = smem + C::kOffK;
+  float* w_s = reinterpret_cast<float*>(smem + C::kOffW);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* acc_empty = acc_full + NUM_ACC;
+  uint64_t* q_full = acc_empty + NUM_ACC;
+  uint64_t* drain_bar = q_full + 1;
+  uint64_t* never_bar = q_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  SelectSmem& sel = *reinterpret_cast<SelectSmem*>(smem + C::kOffSel);
+  uint32_t* sc_s = reinterpret_cast<uint32_t*>(smem + C::kOffScores);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int G = p.G;
+  const int item = blockIdx.x / G;
+  const int b = item % p.B;
+  const int tb = p.ntb - 1 - item / p.B;   // longest (latest) row blocks first
+  const int row0 = tb * NT;
+  const int len = p.lengths[b];
+  const bool bad = len < p.n || len > p.max_len;
+  if (bad && rank == 0 && threadIdx.x == 0) raise_error(p.err, IDX_DEV_ERR_LENGTH);
+
+  int vis[NT];
+  bool exists[NT];
+  int vis_max = 0;
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const int tok = row0 + j;
+    exists[j] = tok < p.n;
+    vis[j] = (exists[j] && !bad) ? (p.causal ? len - p.n + tok + 1 : len) : 0;
+    vis_max = max(vis_max, vis[j]);
+  }
+  const int chunk = vis_max > 0 ? ceil_div(ceil_div(vis_max, G), kTileKeys) * kTileKeys : 0;
+  const int start = static_cast<int>(rank) * chunk;
+  const int end = min(start + chunk, vis_max);
+  const int ntiles = end > start ? ceil_div(end - start, kTileKeys) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < NUM_ACC; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], EPI_WARPS);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(drain_bar, 1);
+    mbar_init(never_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::kTmemCols);
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    const int j = i / IDX_HEADS;
+    const int tok = row0 + j;
+    w_s[i] = (tok < p.n && !bad) ? p.w[(static_cast<int64_t>(b) * p.n + tok) * IDX_HEADS + (i % IDX_HEADS)] : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint64_t budget = p.budget_ns;
+  int tma_issued = 0;   // producer lane: K tiles whose loads were issued
+  bool q_issued = false;  // producer lane: the query load was issued
+  bool mma_issued = false;  // MMA lane: at least one tcgen05.mma issued
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && ntiles > 0) {
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_q);
+      mbar_arrive_expect_tx(q_full, C::kQBytes);
+      tma_load_3d(q_s, &tmap_q, q_full, 0, row0 * IDX_HEADS, b);
+      q_issued = true;
+      int t = 0;
+      for (; t < ntiles; ++t) {
+        const int s = t % STAGES;
+        if (!mbar_wait(&empty[s], ((t / STAGES) & 1) ^ 1, budget, abort_flag, p.err)) break;
+        mbar_arrive_expect_tx(&full[s], kTileBytes);
+        tma_load_3d(k_s + s * kTileBytes, &tmap_k, &full[s], 0, start + t * kTileKeys, b);
+      }
+      tma_issued = t;
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      if (p.debug_flags & 1u) mbar_wait(never_bar, 0, budget, abort_flag, p.err);  // fault injection: nothing arrives
+      if (ntiles > 0 && mbar_wait(q_full, 0, budget, abort_flag, p.err)) {
+        constexpr uint32_t idesc = idesc_e4m3_f32(128, N);
+        const uint32_t q_addr = smem_u32(q_s);
+        for (int t = 0; t < ntiles; ++t) {
+          const int s = t % STAGES;
+          const int a = t % NUM_ACC;
+          if (!mbar_wait(&full[s], (t / STAGES) & 1, budget, abort_flag, p.err)) break;
+          if (!mbar_wait(&acc_empty[a], ((t / NUM_ACC) & 1) ^ 1, budget, abort_flag, p.err)) break;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(k_s + s * kTileBytes);
+          const uint32_t d = tmem_base + static_cast<uint32_t>(a * N);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            mma_e4m3(d, smem_desc_k128_sw128(k_addr + kk * 32), smem_desc_k128_sw128(q_addr + kk * 32), idesc,
+                     kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&acc_full[a]);
+          mma_issued = true;
+        }
+      }
+      if (mma_issued) mma_commit(drain_bar);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;
+    const int quad = warp & 3;                  // TMEM lanes this warp may read
+    const int tok_lo = (ew >> 2) * C::kTokPerWarp;
+    const int kl = quad * 32 + lane;            // key within the tile
+    const float* kscale_row = p.k_scale + static_cast<int64_t>(b) * p.T_cap;
+    for (int t = 0; t < ntiles; ++t) {
+      const int a = t % NUM_ACC;
+      const int key = start + t * kTileKeys + kl;
+      const float ks = key < end ? __ldg(kscale_row + key) : 0.f;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&acc_full[a], (t / NUM_ACC) & 1, budget, abort_flag, p.err) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int jj = 0; jj < C::kTokPerWarp; ++jj) {
+        const int j = tok_lo + jj;
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          float v[32];
+          tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(a * N + j * 64 + c * 32), v);
+          const float4* wv = reinterpret_cast<const float4*>(w_s + j * 64 + c * 32);
+#pragma unroll
+          for (int h4 = 0; h4 < 8; ++h4) {
+            const float4 w4 = wv[h4];
+            part[0] = fmaf(w4.x, fmaxf(v[4 * h4 + 0], 0.f), part[0]);
+            part[1] = fmaf(w4.y, fmaxf(v[4 * h4 + 1], 0.f), part[1]);
+            part[2] = fmaf(w4.z, fmaxf(v[4 * h4 + 2], 0.f), part[2]);
+            part[3] = fmaf(w4.w, fmaxf(v[4 * h4 + 3], 0.f), part[3]);
+          }
+        }
+        const float sc = ((part[0] + part[1]) + (part[2] + part[3])) * ks;
+        if constexpr (FUSED) {
+          sc_s[j * p.chunk_cap + t * kTileKeys + kl] = key < vis[j] ? order_key(sc) : 0u;
+        } else {
+          if (exists[j] && key < p.ld && t * kTileKeys + kl < chunk) {
+            p.scores[(static_cast<int64_t>(b) * p.n + row0 + j) * p.ld + key] = key < vis[j] ? sc : -INFINITY;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[a]);
+    }
+  }
+  __syncthreads();
+
+  if constexpr (!FUSED) {
+    // columns of this CTA's share that no tile covered: −inf
+    const int64_t col_lo = static_cast<int64_t>(start) + static_cast<int64_t>(ntiles) * kTileKeys;
+    const int64_t share_hi = (static_cast<int>(rank) == G - 1) ? p.ld : (p.ld < static_cast<int64_t>(start) + chunk ? p.ld : static_cast<int64_t>(start) + chunk);
+    const int64_t lo = (vis_max == 0 && static_cast<int>(rank) == G - 1) ? 0 : col_lo;
+    if (share_hi > lo) {
+      for (int j = 0; j < NT; ++j) {
+        if (!exists[j]) continue;
+        float* row = p.scores + (static_cast<int64_t>(b) * p.n + row0 + j) * p.ld;
+        for (int64_t c = lo + threadIdx.x; c < share_hi; c += blockDim.x) row[c] = -INFINITY;
+      }
+    }
+  } else {
+    // agree across the cluster on whether anybody gave up
+    cluster_sync();
+    if (threadIdx.x == 0) {
+      int any = 0;
+      for (int r = 0; r < G; ++r) any |= static_cast<int>(dsmem_ld_u32(dsmem_addr((const void*)abort_flag, r)));
+      sel.any_abort = any;
+    }
+    __syncthreads();
+    const bool skip = sel.any_abort != 0;
+    cluster_sync();
+#pragma unroll 1
+    for (int j = 0; j < NT; ++j) {
+      if (!exists[j]) continue;
+      int32_t* out = p.indices + (static_cast<int64_t>(b) * p.n + row0 + j) * p.k;
+      const int v = vis[j];
+      const int kt = min(p.k, v);
+      const int nloc = max(0, min(end, v) - start);
+      if (skip || kt == v) {
+        // every visible position is selected (or the launch gave up): slot s holds position s
+        if (!skip)
+          for (int i = threadIdx.x; i < nloc; i += blockDim.x) out[start + i] = start + i;
+        if (rank == 0)
+          for (int i = (skip ? 0 : kt) + threadIdx.x; i < p.k; i += blockDim.x) out[i] = -1;
+      } else {
+        cluster_select_row(sel, sc_s + j * p.chunk_cap, nloc, start, kt, out, G, rank);
+        if (rank == 0)
+          for (int i = kt + threadIdx.x; i < p.k; i += blockDim.x) out[i] = -1;
+      }
+    }
+    cluster_sync();
+  }
+
+  // ------------------------------------------------------------ teardown
+  if (warp == 0 && lane == 0) {
+    // wait for copies still in flight (bounded) before the CTA's shared memory is released
+    int dummy = 0;
+    if (q_issued) mbar_wait(q_full, 0, budget, &dummy, p.err);
+    for (int t = max(0, tma_issued - STAGES); t < tma_issued; ++t)
+      mbar_wait(&full[t % STAGES], (t / STAGES) & 1, budget, &dummy, p.err);
+  }
+  if (warp == 1 && lane == 0 && mma_issued) {
+    int dummy = 0;
+    mbar_wait(drain_bar, 0, budget, &dummy, p.err);   // all issued MMAs finished
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// ---------------------------------------------------------------- host side
+struct Plan {
+  int G;
+  int chunk_cap;
+  int ntb;
+  int smem;
+};
+
+int pow2_floor(int x) {
+  int p = 1;
+  while (p * 2 <= x) p *= 2;
+  return p;
+}
+
+template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS>
+int launch_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
+                 const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, float* scores,
+                 int64_t ld, int k, int32_t* indices, cudaStream_t stream, int score_budget_bytes) {
+  using C = Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>;
+  const int ntb = (n + NT - 1) / NT;
+  const int64_t items = static_cast<int64_t>(B) * ntb;
+  const int sms = num_sms();
+  // cluster size: enough CTAs to cover the GPU once, and (fused) a score slice that fits
+  int G = 1;
+  if (items < sms) G = pow2_floor(static_cast<int>(sms / items));
+  G = G > 8 ? 8 : G;
+  const int min_keys_per_cta = 512;
+  while (G > 1 && (max_len + G - 1) / G < min_keys_per_cta) G /= 2;
+  auto chunk_of = [&](int g) { return ((max_len + g - 1) / g + kTileKeys - 1) / kTileKeys * kTileKeys; };
+  if (FUSED)
+    while (G < 8 && NT * chunk_of(G) * 4 > score_budget_bytes) G *= 2;
+  const int chunk_cap = chunk_of(G);
+  int smem = C::smem_bytes(FUSED ? chunk_cap : 0);
+  // TMEM has 512 columns per SM and tcgen05.alloc waits for free columns: size the
+  // shared-memory request so that co-resident CTAs never ask for more than 512 in total
+  const int tmem_ctas = 512 / C::kTmemCols;
+  const int per_sm = smem_per_sm();
+  while (per_sm / (smem + 1024) > tmem_ctas) smem += 1024;
+  if (smem > max_dynamic_smem()) return IDX_ERR_SHAPE;
+  if (items * G > 0x7FFFFFFF) return IDX_ERR_SHAPE;
+
+  CUtensorMap tk, tq;
+  if (!make_tmap_u8_3d(&tk, k_cache, IDX_DIM, static_cast<uint64_t>(T_cap), static_cast<uint64_t>(B), kTileKeys))
+    return IDX_ERR_ALIGN;
+  if (!make_tmap_u8_3d(&tq, q_fp8, IDX_DIM, static_cast<uint64_t>(n) * IDX_HEADS, static_cast<uint64_t>(B), C::N))
+    return IDX_ERR_ALIGN;
+
+  auto kern = score_kernel<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>;
+  static int configured_smem = -1;   // per instantiation
+  if (configured_smem < smem) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return check_launch();
+    configured_smem = smem;
+  }
+  ScoreParams p;
+  p.w = w;
+  p.k_scale = k_scale_cache;
+  p.lengths = lengths;
+  p.scores = scores;
+  p.indices = indices;
+  p.ld = ld;
+  p.B = B;
+  p.n = n;
+  p.T_cap = T_cap;
+  p.max_len = max_len;
+  p.causal = causal;
+  p.k = k;
+  p.G = G;
+  p.ntb = ntb;
+  p.chunk_cap = chunk_cap;
+  const DebugState dbg = debug_state();
+  p.debug_flags = dbg.flags;
+  p.budget_ns = dbg.budget_ns;
+  p.err = device_error_word();
+  if (!p.err) return check_launch();
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(items * G), 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(G);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tk, tq, p) != cudaSuccess) return check_launch();
+  return check_launch();
+}
+
+int check_score_args(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
+                     const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal) {
+  if (B < 0 || n < 0 || T_cap <= 0) return IDX_ERR_SHAPE;
+  if (B == 0 || n == 0) return IDX_OK;
+  if (!q_fp8 || !w || !k_cache || !k_scale_cache || !lengths) return IDX_ERR_NULL;
+  if (max_len < n || max_len > T_cap || max_len > IDX_MAX_LEN) return IDX_ERR_SHAPE;
+  if (causal != 0 && causal != 1) return IDX_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(q_fp8) | reinterpret_cast<uintptr_t>(k_cache)) & 15) return IDX_ERR_ALIGN;
+  if (static_cast<int64_t>(n) * IDX_HEADS > 0x7FFFFFFF) return IDX_ERR_SHAPE;
+  return 1;  // proceed
+}
+
+// decode-shaped calls (one or a few rows per sequence) use one row per CTA;
+// prefill-shaped calls four rows (N = 256).
+constexpr int kDecodeRowsMax = 2;
+
+}  // namespace
+
+}  // namespace idx
+
+using namespace idx;
+
+extern "C" int idx_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
+                         const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, float* scores,
+                         int64_t ld, idx_stream_t stream) {
+  const int c = check_score_args(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal);
+  if (c <= 0) return c;
+  if (!scores) return IDX_ERR_NULL;
+  if (ld <= 0) return IDX_ERR_SHAPE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (n <= kDecodeRowsMax)
+    return launch_score<1, false, 8, 4, 4>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
+                                           scores, ld, 0, nullptr, s, 0);
+  return launch_score<4, false, 4, 2, 8>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
+                                         scores, ld, 0, nullptr, s, 0);
+}
+
+extern "C" int idx_score_topk(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache,
+                              const float* k_scale_cache, const int32_t* lengths, int B, int n, int T_cap,
+                              int max_len, int causal, int k, int32_t* indices, void* ws, size_t ws_bytes,
+                              idx_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  const int c = check_score_args(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal);
+  if (c <= 0) return c;
+  if (k <= 0) return IDX_ERR_K;
+  if (!indices) return IDX_ERR_NULL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (n <= kDecodeRowsMax)
+    return launch_score<1, true, 8, 4, 4>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
+                                          nullptr, 0, k, indices, s, 64 * 1024);
+  return launch_score<4, true, 4, 2, 8>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
+                                        nullptr, 0, k, indices, s, 64 * 1024);
+}

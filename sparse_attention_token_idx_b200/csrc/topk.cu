@@ -1,0 +1,115 @@
+// Top-k over scores already in memory (Indexer.forward excerpt: top
+// min(index_topk, ·) positions per row; NKI indexer page: int32, unordered).
+//
+// One thread-block cluster of G CTAs per query row; each CTA loads a
+// contiguous slice of the row's visible scores into shared memory as
+// order-preserving keys, then the cluster runs the same radix select as the
+// fused score kernel.
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "api_internal.h"
+#include "ptx.cuh"
+#include "select.cuh"
+
+namespace idx {
+namespace {
+
+constexpr int kTopkThreads = 256;
+
+struct TopkParams {
+  const float* scores;
+  const int32_t* lengths;
+  int32_t* indices;
+  int64_t ld;
+  int B, n, max_len, causal, k, G, chunk_cap;
+  unsigned int* err;
+};
+
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  SelectSmem& sel = *reinterpret_cast<SelectSmem*>(smem);
+  uint32_t* sc_s = reinterpret_cast<uint32_t*>(smem + sizeof(SelectSmem));
+  const uint32_t rank = cluster_rank();
+  const int G = p.G;
+  const int64_t row = blockIdx.x / G;          // b * n + i
+  const int b = static_cast<int>(row / p.n);
+  const int i = static_cast<int>(row - static_cast<int64_t>(b) * p.n);
+  const int len = p.lengths[b];
+  const bool bad = len < p.n || len > p.max_len;
+  if (bad && rank == 0 && threadIdx.x == 0 && i == 0) raise_error(p.err, IDX_DEV_ERR_LENGTH);
+  const int vis = bad ? 0 : (p.causal ? len - p.n + i + 1 : len);
+  const int chunk = vis > 0 ? (vis + G - 1) / G : 0;
+  const int start = static_cast<int>(rank) * chunk;
+  const int nloc = max(0, min(start + chunk, vis) - start);
+  const float* src = p.scores + row * p.ld + start;
+  for (int t = threadIdx.x; t < nloc; t += blockDim.x) sc_s[t] = order_key(__ldg(src + t));
+  __syncthreads();
+  int32_t* out = p.indices + row * p.k;
+  const int kt = min(p.k, vis);
+  if (kt == vis) {
+    for (int t = threadIdx.x; t < nloc; t += blockDim.x) out[start + t] = start + t;
+  } else {
+    cluster_select_row(sel, sc_s, nloc, start, kt, out, G, rank);
+  }
+  if (rank == 0)
+    for (int t = kt + threadIdx.x; t < p.k; t += blockDim.x) out[t] = -1;
+  cluster_sync();
+}
+
+int pow2_floor_i(int x) {
+  int r = 1;
+  while (r * 2 <= x) r *= 2;
+  return r;
+}
+
+}  // namespace
+}  // namespace idx
+
+using namespace idx;
+
+extern "C" int idx_topk(const float* scores, const int32_t* lengths, int B, int n, int64_t ld, int max_len,
+                        int causal, int k, int32_t* indices, void* ws, size_t ws_bytes, idx_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (B < 0 || n < 0) return IDX_ERR_SHAPE;
+  if (k <= 0) return IDX_ERR_K;
+  if (B == 0 || n == 0) return IDX_OK;
+  if (!scores || !lengths || !indices) return IDX_ERR_NULL;
+  if (causal != 0 && causal != 1) return IDX_ERR_SHAPE;
+  if (max_len < n || max_len > IDX_MAX_LEN || static_cast<int64_t>(max_len) > ld) return IDX_ERR_SHAPE;
+  const int64_t rows = static_cast<int64_t>(B) * n;
+  const int sms = num_sms();
+  int G = rows < sms ? pow2_floor_i(static_cast<int>(sms / rows)) : 1;
+  if (G > 8) G = 8;
+  while (G > 1 && (max_len + G - 1) / G < 512) G /= 2;
+  const int budget = 64 * 1024;
+  while (G < 8 && static_cast<int64_t>((max_len + G - 1) / G) * 4 > budget) G *= 2;
+  const int chunk_cap = (max_len + G - 1) / G;
+  const int smem = 128 + static_cast<int>(sizeof(SelectSmem)) + chunk_cap * 4;
+  if (smem > max_dynamic_smem()) return IDX_ERR_SHAPE;
+  if (rows * G > 0x7FFFFFFF) return IDX_ERR_SHAPE;
+  static int configured = -1;
+  if (configured < smem) {
+    if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return check_launch();
+    configured = smem;
+  }
+  TopkParams p{scores, lengths, indices, ld, B, n, max_len, causal, k, G, chunk_cap, device_error_word()};
+  if (!p.err) return check_launch();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows * G), 1, 1);
+  cfg.blockDim = dim3(kTopkThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(G);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, topk_kernel, p);
+  return check_launch();
+}

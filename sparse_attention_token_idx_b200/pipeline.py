@@ -1,0 +1,45 @@
+"""One indexer call on the GPU, in the order the reference forward takes:
+append this call's keys to the cache, quantise the queries and fold the head
+weights, then score every query row against the cache and select its top-k.
+
+``Indexer`` owns the cache buffers (kept between calls) and the per-call
+scratch tensors; every step runs in libidx.so through ``binding``.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as X
+
+
+class Indexer:
+    def __init__(self, B: int, T_cap: int, fmt: int, k: int, device="cuda"):
+        self.B, self.T_cap, self.fmt, self.k = B, T_cap, fmt, k
+        self.device = torch.device(device)
+        self.k_cache = torch.zeros((B, T_cap, X.DIM), dtype=torch.uint8, device=self.device)
+        self.k_scale_cache = torch.zeros((B, T_cap), dtype=torch.float32, device=self.device)
+        self._bufs = {}
+
+    def _buf(self, name, shape, dtype):
+        t = self._bufs.get(name)
+        if t is None or t.shape != shape or t.dtype != dtype:
+            t = torch.empty(shape, dtype=dtype, device=self.device)
+            self._bufs[name] = t
+        return t
+
+    def append(self, k_new: torch.Tensor, positions: torch.Tensor, stream=None):
+        """Rotate, quantise and store k_new [B, n, 128] bf16 at slots positions[b] …"""
+        X.quant_append(k_new, positions, self.k_cache, self.k_scale_cache, self.fmt, stream=stream)
+
+    def step(self, k_new, q, w_raw, positions, lengths, *, causal: bool, max_len: int, out=None, stream=None):
+        """k_new [B, n, 128] bf16, q [B, n, 64, 128] bf16, w_raw [B, n, 64] fp32,
+        positions [B] int32 (first new slot), lengths [B] int32 (= positions + n),
+        max_len ≥ max(lengths) on the host.  Returns top-k positions [B, n, k] int32."""
+        B, n = q.shape[0], q.shape[1]
+        self.append(k_new, positions, stream=stream)
+        q_fp8 = self._buf("q_fp8", tuple(q.shape), torch.uint8)
+        w = self._buf("w", tuple(w_raw.shape), torch.float32)
+        X.quant_queries(q, w_raw, self.fmt, q_out=q_fp8, w_out=w, stream=stream)
+        out = out if out is not None else self._buf("idx", (B, n, self.k), torch.int32)
+        return X.score_topk(q_fp8, w, self.k_cache, self.k_scale_cache, lengths, causal, self.k, max_len,
+                            out=out, stream=stream)

@@ -1,0 +1,58 @@
+"""CPU-side checks of the boundary: the shared library builds, loads without a
+GPU, exports exactly the functions include/idx.h declares, and the binding's
+signatures cover them; the product path raises when no GPU is present."""
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "idx.h")).read()
+    return set(re.findall(r"IDX_API\s+[\w\s\*]+?\b(idx_\w+)\s*\(", src))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ["idx_quant", "idx_quant_append", "idx_score", "idx_topk", "idx_score_topk", "idx_workspace_size",
+              "idx_status", "idx_error_string"]:
+        assert n in names
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    from sparse_attention_token_idx_b200 import binding, build
+    build.build()
+    lib = binding.load()
+    for n in _declared():
+        assert hasattr(lib, n), n
+    assert set(binding.SIGNATURES) == _declared()
+
+
+def test_error_strings_without_gpu():
+    from sparse_attention_token_idx_b200 import binding
+    lib = binding.load()
+    assert lib.idx_error_string(0) == b"ok"
+    assert b"NULL" in lib.idx_error_string(-1)
+    assert lib.idx_workspace_size(128, 1, 16384, 2048) == 0
+
+
+def test_host_argument_checks_run_before_any_device_work():
+    from sparse_attention_token_idx_b200 import binding
+    lib = binding.load()
+    # rejected on the host: nothing touches the (absent) GPU
+    assert lib.idx_quant(None, 0, None, None, 7, None) == -3
+    assert lib.idx_quant(None, 5, None, None, 0, None) == -1
+    assert lib.idx_score_topk(None, None, None, None, None, 1, 1, 16, 16, 0, 0, None, None, 0, None) == -1
+    assert lib.idx_topk(None, None, 1, 1, 16, 16, 0, 0, None, None, 0, None) == -4
+    assert lib.idx_quant_append(None, None, -1, 1, None, None, 16, 0, None) == -2
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_product_path_fails_loudly_without_gpu():
+    from sparse_attention_token_idx_b200 import binding
+    x = torch.zeros((4, 128), dtype=torch.bfloat16)
+    with pytest.raises(binding.IdxError):
+        binding.quant(x, 0)

@@ -1,0 +1,75 @@
+"""Standalone top-k (idx_topk) on exactly known scores, and the fused
+score + top-k (idx_score_topk) against the oracle and against idx_score."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import indexer as O
+from sparse_attention_token_idx_b200 import synth
+from tests.helpers import (check_topk_exact_row, check_topk_row, dev, gpu_queries, gpu_state, oracle_queries,
+                           oracle_state)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("B,n,lengths,causal,k,ties", [
+    (4, 1, [1, 2047, 2049, 16384], False, 2048, False),
+    (3, 1, [5000, 9000, 3000], False, 100, True),      # heavy ties at the threshold
+    (1, 1, [131072], False, 2048, False),               # longest row: full cluster
+    (2, 40, [40, 3000], True, 64, True),
+    (16, 1, list(range(1000, 17000, 1000)), False, 2048, True),
+])
+def test_topk_exact(B, n, lengths, causal, k, ties):
+    from sparse_attention_token_idx_b200 import binding as X
+    rng = np.random.default_rng(sum(lengths) + k)
+    ld = max(lengths)
+    sc = rng.standard_normal((B, n, ld)).astype(np.float32)
+    if ties:
+        sc = np.round(sc * 8) / 8                     # a few hundred distinct values
+    sc[:, :, ::97] = -sc[:, :, ::97] * 1e30           # very large magnitudes of both signs
+    lengths = np.array(lengths, np.int32)
+    got = X.topk(dev(sc), dev(lengths), causal, k, ld).cpu().numpy()
+    assert X.status() == (0, 0)
+    for b in range(B):
+        for i in range(n):
+            vis = O.visible_count(int(lengths[b]), n, i, causal)
+            check_topk_exact_row(got[b, i], sc[b, i], vis, k)
+
+
+def test_topk_negative_zero_and_infinities():
+    from sparse_attention_token_idx_b200 import binding as X
+    s = np.array([[[0.0, -0.0, 1.0, -np.inf, np.inf, -1.0, 0.0, -0.0]]], np.float32)
+    got = X.topk(dev(s), dev(np.array([8], np.int32)), False, 5, 8).cpu().numpy()
+    # +inf, 1.0, then three of the four zeros (−0 and +0 compare equal as scores)
+    sel = set(got[0, 0].tolist())
+    assert {4, 2} <= sel and len(sel) == 5 and sel - {4, 2} <= {0, 1, 6, 7}
+
+
+FUSED = [
+    ("decode-mixed", 6, 1, [0, 100, 2046, 2048, 5000, 16383], 16384, False, 0, 2048),
+    ("decode-single", 1, 1, [4095], 4096, False, 1, 2048),
+    ("decode-small-k", 4, 1, [511, 2000, 777, 3333], 4096, False, 0, 17),
+    ("prefill", 1, 300, [0], 512, True, 0, 64),
+    ("chunked", 2, 130, [900, 2500], 4096, True, 1, 512),
+]
+
+
+@pytest.mark.parametrize("name,B,n,positions,T_cap,causal,fmt,k", FUSED)
+def test_fused_topk_matches_oracle_and_unfused(name, B, n, positions, T_cap, causal, fmt, k):
+    from sparse_attention_token_idx_b200 import binding as X
+    case = synth.make_case(name, 300 + len(name), B, n, positions, T_cap=T_cap, causal=causal, fmt=fmt, k=k)
+    kc, ks, lengths = gpu_state(case)
+    qc, w = gpu_queries(case)
+    max_len = int(case.lengths.max())
+    idx = X.score_topk(qc, w, kc, ks, lengths, causal, k, max_len).cpu().numpy()
+    sc = X.score(qc, w, kc, ks, lengths, causal, max_len, ld=max_len).cpu().numpy()
+    assert X.status() == (0, 0)
+    okc, oks = oracle_state(case)
+    oqc, ow = oracle_queries(case)
+    S, E = O.index_scores(oqc, ow, okc, oks, case.lengths, causal, ncols=max_len)
+    for b in range(B):
+        for i in range(n):
+            vis = O.visible_count(int(case.lengths[b]), n, i, causal)
+            check_topk_row(idx[b, i], S[b, i], E[b, i], vis, k)
+            # the fused kernel selects from the very fp32 scores idx_score writes
+            check_topk_exact_row(idx[b, i], sc[b, i], vis, k)
