@@ -1,0 +1,450 @@
+"""Benchmark of the lightning-indexer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl ours|reference]
+
+A step is one whole indexer call on one batch: append the new keys to the FP8
+cache (rotate + quantise + store), quantise the queries and fold the head
+weights, then the fused score + top-k over every cached key.  The default
+workload is the bandwidth-bound decode case (B = 128 sequences, 16 384 cached
+keys each, ue8m0 scales, k = 2048): its 277 MB FP8 cache is larger than the
+126 MB L2, so consecutive steps stream it from HBM.  Other workloads
+(--workload 0…4) are for measurement notes; the prefill ones report FP8
+TFLOP/s.
+
+Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
+sequences (weak scaling, no data-path collective); times are the max over
+ranks.  ``--impl reference`` times the CPU oracle (the only reference
+implementation there is) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = 2
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP8_PER_BF16 = 2.0            # nominal dense fp8 : bf16 tensor ratio on B200
+KEY_BYTES = 128 + 4           # one cached key: 128 e4m3 codes + fp32 scale
+ROW_BYTES_IN = 64 * 128 + 64 * 4   # one query row: 64 heads of e4m3 codes + 64 fp32 weights
+PROFILE_SCORE = os.path.join(ROOT, "profiles", "score_topk_decode_b128_t16384.md")
+KERNEL_SOURCES = ["score.cu", "select.cuh", "ptx.cuh"]
+
+
+def env_rank():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return d.get("hbm_gbs"), d.get("bf16_tflops"), d.get("bf16_tflops_sustained"), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "sparse_attention_token_idx_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(path, launch_units):
+    """DRAM bytes per launch from a committed ncu summary, scaled to this launch's
+    units, or None when the summary is missing or the kernel source changed."""
+    try:
+        kv = {}
+        for line in open(path):
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                kv[k.strip()] = v.strip().strip("`")
+        if kv.get("source_sha256") != kernel_source_hash():
+            return None
+        per_unit = float(kv["dram_bytes_per_key"])
+        return per_unit * launch_units
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = [name for bit, name in self.REASONS.items() if self.reasons & bit and bit != 0x1]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------- workload
+def workload_numbers(case):
+    """Algorithmic per-step units: keys scored, bytes the fused kernel must move, FLOPs."""
+    n = case.n
+    keys = 0
+    for b in range(case.B):
+        L = int(case.lengths[b])
+        if case.causal:
+            keys += int(np.arange(L - n + 1, L + 1).sum())    # row i sees L - n + i + 1 keys
+        else:
+            keys += L * n
+    flops = 2 * 64 * 128 * keys
+    key_rows = int(case.lengths.sum())                  # each cached key read once per launch
+    rows = case.B * n
+    score_bytes = key_rows * KEY_BYTES + rows * (ROW_BYTES_IN + 4 * case.k) + case.B * 4
+    return keys, flops, key_rows, score_bytes
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from sparse_attention_token_idx_b200 import binding as X
+    from sparse_attention_token_idx_b200 import synth
+    from sparse_attention_token_idx_b200.pipeline import Indexer
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    case = synth.workload(args.workload)
+    B, n = case.B, case.n
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    dv = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    ix = Indexer(B, case.T_cap, case.fmt, case.k, device=dev)
+    P = case.k_prior.shape[1]
+    if P:
+        if np.all(case.positions == P):
+            ix.append(bf(case.k_prior), dv(np.zeros(B, np.int32)))
+        else:
+            for b in range(B):
+                p = int(case.positions[b])
+                if p:
+                    X.quant_append(bf(case.k_prior[b:b + 1, :p]), dv(np.zeros(1, np.int32)), ix.k_cache[b:b + 1],
+                                   ix.k_scale_cache[b:b + 1], case.fmt)
+    k_new, q, w_raw = bf(case.k_new), bf(case.q), dv(case.w_raw)
+    positions, lengths = dv(case.positions), dv(case.lengths)
+    max_len = int(case.lengths.max())
+    out = torch.empty((B, n, case.k), dtype=torch.int32, device=dev)
+    q_fp8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
+    w = torch.empty(w_raw.shape, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    keys, flops, key_rows, score_bytes = workload_numbers(case)
+
+    def step(ev=None):
+        ix.append(k_new, positions)
+        X.quant_queries(q, w_raw, case.fmt, q_out=q_fp8, w_out=w)
+        if ev is not None:
+            ev[0].record(stream)
+        X.score_topk(q_fp8, w, ix.k_cache, ix.k_scale_cache, lengths, case.causal, case.k, max_len, out=out)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    code, bits = X.status()
+    if code != 0:
+        raise RuntimeError(f"device error during warm-up: status {code}, bits {bits}")
+
+    # -------------------------------------------------------------- timed region
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    with sampler:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    score_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    code, bits = X.status()
+    if code != 0:
+        raise RuntimeError(f"device error in the timed region: status {code}, bits {bits}")
+
+    # -------------------------------------------------------------- end to end from pinned host memory
+    h_k = case_pinned(torch, case.k_new.view(np.int16)).view(torch.bfloat16)
+    h_q = case_pinned(torch, case.q.view(np.int16)).view(torch.bfloat16)
+    h_w = case_pinned(torch, case.w_raw)
+    h_p = case_pinned(torch, case.positions)
+    h_l = case_pinned(torch, case.lengths)
+    h_out = torch.empty((B, n, case.k), dtype=torch.int32).pin_memory()
+    d_k, d_q, d_w = torch.empty_like(k_new), torch.empty_like(q), torch.empty_like(w_raw)
+    d_p, d_l = torch.empty_like(positions), torch.empty_like(lengths)
+    h2d = sum(t.numel() * t.element_size() for t in (h_k, h_q, h_w, h_p, h_l))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def step_e2e():
+        d_k.copy_(h_k, non_blocking=True)
+        d_q.copy_(h_q, non_blocking=True)
+        d_w.copy_(h_w, non_blocking=True)
+        d_p.copy_(h_p, non_blocking=True)
+        d_l.copy_(h_l, non_blocking=True)
+        idx = ix.step(d_k, d_q, d_w, d_p, d_l, causal=case.causal, max_len=max_len)
+        h_out.copy_(idx, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 2000))
+    for _ in range(args.warmup):
+        step_e2e()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        step_e2e()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    code, bits = X.status()
+    if code != 0:
+        raise RuntimeError(f"device error in the end-to-end loop: status {code}, bits {bits}")
+
+    # -------------------------------------------------------------- reduce over ranks (max time)
+    t = torch.tensor([ms, score_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, score_ms, e2e_ms = t.tolist()
+    return dict(case=case, keys=keys, flops=flops, key_rows=key_rows, score_bytes=score_bytes, ms=ms,
+                score_ms=score_ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
+                clocks=sampler.summary(), launches=3 * args.steps)
+
+
+def case_pinned(torch, a):
+    return torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+
+
+# ---------------------------------------------------------------------------- oracle timing
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_step_timer(case, seqs, key_limit=None):
+    """Build the oracle's cache for ``seqs`` (untimed) and return a function that
+    runs one oracle step on them (append this call's keys, quantise queries,
+    fp64 scores, full-sort top-k) and the keys it scores."""
+    from oracle import indexer as O
+    B, n = case.B, case.n
+    kc = np.zeros((B, case.T_cap, 128), np.uint8)
+    ks = np.zeros((B, case.T_cap), np.float32)
+    for b in seqs:
+        p = int(case.positions[b])
+        lim = p if key_limit is None else min(p, key_limit)
+        if lim:
+            O.quant_append(case.k_prior[b:b + 1, :lim], [0], kc[b:b + 1], ks[b:b + 1], case.fmt)
+    lengths = case.lengths.copy()
+    positions = case.positions.copy()
+    if key_limit is not None:
+        positions = np.minimum(positions, key_limit)
+        lengths = positions + n
+    sel = list(seqs)
+
+    def run():
+        st = {"k_cache": kc[sel], "k_scale_cache": ks[sel]}
+        O.indexer_step(st, case.k_new[sel], case.q[sel], case.w_raw[sel], positions[sel], case.causal, case.k,
+                       case.fmt)
+
+    if case.causal:
+        keys = sum(int(((np.arange(lengths[b] - n + 1, lengths[b] + 1)).sum())) for b in sel)
+    else:
+        keys = sum(int(lengths[b]) * n for b in sel)
+    return run, keys
+
+
+def cpu_baseline(case, target_s=8.0, max_seqs=64):
+    """Time the oracle on a bounded sample of the workload, scaled to keys/s."""
+    seqs = [0]
+    run, keys = oracle_step_timer(case, seqs)
+    t = time.perf_counter()
+    run()
+    one = time.perf_counter() - t
+    nseq = int(max(1, min(case.B, max_seqs, target_s / max(one, 1e-3))))
+    if nseq > 1:
+        seqs = list(range(nseq))
+        run, keys = oracle_step_timer(case, seqs)
+    t = time.perf_counter()
+    run()
+    dt = time.perf_counter() - t
+    return {"value": keys / dt, "unit": "keys/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{len(seqs)} of {case.B} sequences of '{case.name}', one full oracle step "
+                      f"(append, quantise queries, fp64 scores, full-sort top-{case.k}) in {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    from sparse_attention_token_idx_b200 import synth
+    case = synth.workload(args.workload)
+    budget_s = 150.0
+    per_step = budget_s / max(1, args.steps + args.warmup)
+    # size each step: one sequence, its first `limit` cached keys, so the whole run stays bounded
+    run, keys = oracle_step_timer(case, [0])
+    t = time.perf_counter()
+    run()
+    full = time.perf_counter() - t
+    limit = None
+    if full > per_step:
+        limit = max(128, int(int(case.positions[0]) * per_step / full))
+        run, keys = oracle_step_timer(case, [0], key_limit=limit)
+    for _ in range(args.warmup):
+        run()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t
+    value = keys * args.steps / dt
+    sample = (f"1 of {case.B} sequences of '{case.name}' per step"
+              + (f", its first {limit} cached keys" if limit else "") + ", full oracle step")
+    return case, value, dt, sample
+
+
+# ---------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    rank, world, local_rank = env_rank()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        case, value, dt, sample = run_reference(args, rank, world)
+        unit = "keys/s"
+        line = {"metric": metric_name(case), "value": value, "unit": unit, "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "impl": "reference",
+                "config": {"workload": case.name, "B": case.B, "n": case.n, "T_cap": case.T_cap, "k": case.k},
+                "cpu_baseline": {"value": value, "unit": unit, "cores": oracle_threads(), "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+    try:
+        r = run_ours(args, rank, world, local_rank)
+    finally:
+        pass
+    case = r["case"]
+    hbm, bf16, bf16_sus, peak_src = measured_peaks()
+    step_s = r["ms"] / 1e3 / args.steps
+    value = r["keys"] * world / step_s
+    e2e_value = r["keys"] * world / (r["e2e_ms"] / 1e3 / r["e2e_steps"])
+    score_s = r["score_ms"] / 1e3
+    if case.causal:
+        achieved = r["flops"] / score_s / 1e12
+        peak = bf16 * FP8_PER_BF16
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": None, "peak_source": f"{peak_src} bf16 burst x nominal fp8/bf16 ratio {FP8_PER_BF16}",
+                "kernel": "score_topk"}
+    else:
+        achieved = r["score_bytes"] / score_s / 1e9
+        traffic = profile_traffic(PROFILE_SCORE, r["key_rows"]) if args.workload == DEFAULT_WORKLOAD else None
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": traffic, "peak_source": f"{peak_src} copy bandwidth", "kernel": "score_topk",
+                "kernel_us": r["score_ms"] * 1e3, "algorithmic_bytes": r["score_bytes"]}
+    line = {
+        "metric": metric_name(case), "value": value, "unit": "keys/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8-e4m3 x fp8-e4m3 -> fp32", "data": "synthetic",
+        "config": {"workload": case.name, "B": case.B, "n": case.n, "T_cap": case.T_cap, "k": case.k,
+                   "heads": 64, "head_dim": 128, "fmt": ["fp32", "ue8m0"][case.fmt],
+                   "l2": ("inputs larger than L2: %.0f MB FP8 cache streamed per step" % (r["key_rows"] * KEY_BYTES / 1e6))
+                   if r["key_rows"] * KEY_BYTES > 126e6 else "L2-resident working set (not flushed)",
+                   "parallelism": f"dp{world} (independent sequences per rank)"},
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": "keys/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "steps": r["e2e_steps"]},
+        "gpu_launches": r["launches"],
+        "clocks": r["clocks"],
+    }
+    if case.causal:
+        line["tflops"] = r["flops"] * world / step_s / 1e12
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case)
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def metric_name(case):
+    return "prefill keys scored+top-k/s (FP8 TFLOP/s in tflops)" if case.causal else "decode keys scored+top-k/s"
+
+
+if __name__ == "__main__":
+    main()

@@ -177,6 +177,16 @@ IDX_API int idx_e4m3_encode(const float* x, int64_t count, uint8_t* out, idx_str
  */
 IDX_API void idx_debug_set(unsigned int flags, unsigned long long budget_ns);
 
+/*
+ * Profiling aid: when the debug flags have bit 1 set, score launches record per
+ * CTA (first 8192 CTAs) 16 words: [0] entry, [1] set-up done, [2] first
+ * accumulator ready, [3] key stream done, [4] selection done, [5] exit
+ * (globaltimer ns), [7] SM id, [8..14] steps inside the first row's
+ * selection, [15] its candidate count.  idx_debug_trace copies them to
+ * host_out (max_ctas × 16 words) after synchronising the device.
+ */
+IDX_API int idx_debug_trace(unsigned long long* host_out, int max_ctas);
+
 #ifdef __cplusplus
 }
 #endif

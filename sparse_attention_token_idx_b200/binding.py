@@ -44,6 +44,7 @@ SIGNATURES = {
     "idx_last_cuda_error": (_I, []),
     "idx_e4m3_encode": (_I, [_P, _I64, _P, _P]),
     "idx_debug_set": (None, [ctypes.c_uint, ctypes.c_ulonglong]),
+    "idx_debug_trace": (_I, [_P, _I]),
 }
 
 _lib = None
@@ -182,3 +183,11 @@ def status(stream=None) -> tuple[int, int]:
 
 def debug_set(flags: int, budget_ns: int = 0):
     load().idx_debug_set(flags, budget_ns)
+
+
+def debug_trace(max_ctas: int):
+    """Per-CTA phase timestamps of the last traced score launch (see include/idx.h)."""
+    import numpy as np
+    buf = np.zeros((max_ctas, 16), np.uint64)
+    _check(load().idx_debug_trace(buf.ctypes.data, max_ctas), "idx_debug_trace")
+    return buf

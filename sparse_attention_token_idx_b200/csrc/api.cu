@@ -98,8 +98,7 @@ int check_launch() {
                                                                                        : IDX_ERR_LAUNCH;
 }
 
-bool make_tmap_u8_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
-                     uint32_t box_rows) {
+static void resolve_encode() {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -107,6 +106,11 @@ bool make_tmap_u8_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_
         q == cudaDriverEntryPointSuccess)
       g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   });
+}
+
+bool make_tmap_u8_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                     uint32_t box_rows) {
+  resolve_encode();
   if (!g_encode) return false;
   if (reinterpret_cast<uintptr_t>(base) & 15) return false;
   const cuuint64_t dims[3] = {inner, mid, outer};
@@ -115,6 +119,20 @@ bool make_tmap_u8_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner) {
+  resolve_encode();
+  if (!g_encode) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((inner * 4) & 15)) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 4};
+  const cuuint32_t box[2] = {box_inner, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }

@@ -20,6 +20,12 @@ bool make_tmap_u8_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_
 
 unsigned int* device_error_word();  // device address of the error word on the current device
 
+// Tensor map for a [outer, inner] float32 array (row pitch inner·4 bytes, a
+// multiple of 16), box {box_inner, 1}, no swizzle.
+bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner);
+
+unsigned long long* trace_buffer();  // device address of the phase-trace buffer
+
 struct DebugState {
   unsigned int flags;
   unsigned long long budget_ns;

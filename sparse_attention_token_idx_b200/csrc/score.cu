@@ -28,6 +28,12 @@
 
 namespace idx {
 
+// Phase timestamps per CTA (globaltimer, ns), written only when the trace flag
+// (bit 1 of the debug flags) is set; read back with idx_debug_trace().
+constexpr int kTraceCtas = 8192;
+constexpr int kTraceSlots = 16;
+__device__ unsigned long long g_trace[kTraceCtas * kTraceSlots];
+
 namespace {
 
 constexpr int kTileKeys = 128;
@@ -49,7 +55,7 @@ struct ScoreParams {
   unsigned int* err;         // device error word
 };
 
-template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS>
+template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT>
 struct Cfg {
   static constexpr int N = NT * IDX_HEADS;
   static constexpr int kThreads = (2 + EPI_WARPS) * 32;
@@ -57,18 +63,25 @@ struct Cfg {
   static constexpr int kTmemCols = kAccCols <= 32 ? 32 : kAccCols <= 64 ? 64 : kAccCols <= 128 ? 128
                                  : kAccCols <= 256 ? 256 : 512;
   static_assert(kAccCols <= 512, "TMEM holds 512 columns");
-  static_assert(EPI_WARPS % 4 == 0 && NT % (EPI_WARPS / 4) == 0, "epilogue split");
-  static constexpr int kTokPerWarp = NT / (EPI_WARPS / 4);
+  // epilogue warps: 4 TMEM lane quadrants × token groups × tile phases (TSPLIT)
+  static constexpr int kTokGroups = EPI_WARPS / 4 / TSPLIT;
+  static_assert(EPI_WARPS % (4 * TSPLIT) == 0 && NT % kTokGroups == 0, "epilogue split");
+  static constexpr int kTokPerWarp = NT / kTokGroups;
+  static constexpr int kWarpsPerTile = EPI_WARPS / TSPLIT;   // warps that consume one tile
   static constexpr int kQBytes = N * IDX_DIM;
+  static constexpr int kCand = NT == 1 ? 4096 : 1024;     // candidate list of the select
   // shared memory carve (offsets from a 1024-aligned base)
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffW = kOffK + STAGES * kTileBytes;
+  static constexpr int kOffScale = kOffK + STAGES * kTileBytes;
+  static constexpr int kOffW = kOffScale + STAGES * kTileKeys * 4;
   static constexpr int kOffBar = kOffW + N * 4;
   static constexpr int kNumBars = 2 * STAGES + 2 * NUM_ACC + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffSel = (kOffMisc + 64 + 127) / 128 * 128;
-  static constexpr int kOffScores = kOffSel + (FUSED ? static_cast<int>(sizeof(SelectSmem)) : 0);
+  static constexpr int kOffHist1 = kOffSel + (FUSED ? static_cast<int>(sizeof(SelectSmem)) : 0);
+  static constexpr int kOffCand = kOffHist1 + (FUSED ? NT * kHistBins * 4 : 0);
+  static constexpr int kOffScores = kOffCand + (FUSED ? kCand * 4 : 0);
   static int smem_bytes(int chunk_cap) {
     return 1024 + kOffScores + (FUSED ? NT * chunk_cap * 4 : 0);
   }
@@ -76,16 +89,18 @@ struct Cfg {
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS>
-__global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>::kThreads, 1)
+template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT>
+__global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT>::kThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
-                 const ScoreParams p) {
-  using C = Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>;
+                 const __grid_constant__ CUtensorMap tmap_s, const ScoreParams p) {
+  using C = Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT>;
   constexpr int N = C::N;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base (128-byte swizzle atoms), kept as a shared-space pointer
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* q_s = smem + C::kOffQ;
   uint8_t* k_s = smem + C::kOffK;
+  float* scale_s = reinterpret_cast<float*>(smem + C::kOffScale);
   float* w_s = reinterpret_cast<float*>(smem + C::kOffW);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;
@@ -98,10 +113,20 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>::kT
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   SelectSmem& sel = *reinterpret_cast<SelectSmem*>(smem + C::kOffSel);
+  uint32_t* hist1 = reinterpret_cast<uint32_t*>(smem + C::kOffHist1);
+  int* cand = reinterpret_cast<int*>(smem + C::kOffCand);
   uint32_t* sc_s = reinterpret_cast<uint32_t*>(smem + C::kOffScores);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const bool trace = (p.debug_flags & 2u) && blockIdx.x < kTraceCtas;
+  unsigned long long* tr = g_trace + static_cast<size_t>(blockIdx.x) * kTraceSlots;
+  if (trace && threadIdx.x == 0) {
+    unsigned int smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    tr[0] = globaltimer_ns();
+    tr[7] = smid;
+  }
   const uint32_t rank = cluster_rank();
   const int G = p.G;
   const int item = blockIdx.x / G;
@@ -130,11 +155,11 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>::kT
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 1 + C::kWarpsPerTile);   // MMA done with the keys, epilogue with the scales
     }
     for (int a = 0; a < NUM_ACC; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], EPI_WARPS);
+      mbar_init(&acc_empty[a], C::kWarpsPerTile);
     }
     mbar_init(q_full, 1);
     mbar_init(drain_bar, 1);
@@ -148,11 +173,14 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>::kT
     const int tok = row0 + j;
     w_s[i] = (tok < p.n && !bad) ? p.w[(static_cast<int64_t>(b) * p.n + tok) * IDX_HEADS + (i % IDX_HEADS)] : 0.f;
   }
+  if constexpr (FUSED)
+    for (int i = threadIdx.x; i < NT * kHistBins; i += blockDim.x) hist1[i] = 0;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint64_t budget = p.budget_ns;
+  if (trace && threadIdx.x == 0) tr[1] = globaltimer_ns();
   int tma_issued = 0;   // producer lane: K tiles whose loads were issued
   bool q_issued = false;  // producer lane: the query load was issued
   bool mma_issued = false;  // MMA lane: at least one tcgen05.mma issued
@@ -162,6 +190,7 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>::kT
     if (lane == 0 && ntiles > 0) {
       tma_prefetch_desc(&tmap_k);
       tma_prefetch_desc(&tmap_q);
+      tma_prefetch_desc(&tmap_s);
       mbar_arrive_expect_tx(q_full, C::kQBytes);
       tma_load_3d(q_s, &tmap_q, q_full, 0, row0 * IDX_HEADS, b);
       q_issued = true;
@@ -169,8 +198,9 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>::kT
       for (; t < ntiles; ++t) {
         const int s = t % STAGES;
         if (!mbar_wait(&empty[s], ((t / STAGES) & 1) ^ 1, budget, abort_flag, p.err)) break;
-        mbar_arrive_expect_tx(&full[s], kTileBytes);
+        mbar_arrive_expect_tx(&full[s], kTileBytes + kTileKeys * 4);
         tma_load_3d(k_s + s * kTileBytes, &tmap_k, &full[s], 0, start + t * kTileKeys, b);
+        tma_load_2d(scale_s + s * kTileKeys, &tmap_s, &full[s], start + t * kTileKeys, b);
       }
       tma_issued = t;
     }
@@ -207,51 +237,84 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>::kT
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
     const int quad = warp & 3;                  // TMEM lanes this warp may read
-    const int tok_lo = (ew >> 2) * C::kTokPerWarp;
+    const int tphase = (ew >> 2) % TSPLIT;      // this warp takes tiles t ≡ tphase (mod TSPLIT)
+    const int tok_lo = ((ew >> 2) / TSPLIT) * C::kTokPerWarp;
     const int kl = quad * 32 + lane;            // key within the tile
-    const float* kscale_row = p.k_scale + static_cast<int64_t>(b) * p.T_cap;
-    for (int t = 0; t < ntiles; ++t) {
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    float wreg[C::kTokPerWarp == 1 ? 64 : 1];
+    if constexpr (C::kTokPerWarp == 1) {
+#pragma unroll
+      for (int h = 0; h < 64; ++h) wreg[h] = w_s[tok_lo * 64 + h];
+    }
+    for (int t = tphase; t < ntiles; t += TSPLIT) {
       const int a = t % NUM_ACC;
+      const int s = t % STAGES;
       const int key = start + t * kTileKeys + kl;
-      const float ks = key < end ? __ldg(kscale_row + key) : 0.f;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&acc_full[a], (t / NUM_ACC) & 1, budget, abort_flag, p.err) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
+      if (trace && t == 0 && ew == 0 && lane == 0) tr[2] = globaltimer_ns();
       tc_fence_after();
+      const float ks = scale_s[s * kTileKeys + kl];   // landed with the keys (same barrier)
 #pragma unroll
       for (int jj = 0; jj < C::kTokPerWarp; ++jj) {
         const int j = tok_lo + jj;
+        uint32_t r0[32], r1[32];
+        tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64), r0);
+        tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64 + 32), r1);
+        tmem_wait();
+        tmem_regs_ready(r0);
+        tmem_regs_ready(r1);
         float part[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (C::kTokPerWarp == 1) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float v[32];
-          tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(a * N + j * 64 + c * 32), v);
-          const float4* wv = reinterpret_cast<const float4*>(w_s + j * 64 + c * 32);
+          for (int h = 0; h < 32; ++h)
+            part[h & 3] = fmaf(wreg[h], fmaxf(__uint_as_float(r0[h]), 0.f), part[h & 3]);
+#pragma unroll
+          for (int h = 0; h < 32; ++h)
+            part[h & 3] = fmaf(wreg[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), part[h & 3]);
+        } else {
+          const float4* wv = reinterpret_cast<const float4*>(w_s + j * 64);
 #pragma unroll
           for (int h4 = 0; h4 < 8; ++h4) {
             const float4 w4 = wv[h4];
-            part[0] = fmaf(w4.x, fmaxf(v[4 * h4 + 0], 0.f), part[0]);
-            part[1] = fmaf(w4.y, fmaxf(v[4 * h4 + 1], 0.f), part[1]);
-            part[2] = fmaf(w4.z, fmaxf(v[4 * h4 + 2], 0.f), part[2]);
-            part[3] = fmaf(w4.w, fmaxf(v[4 * h4 + 3], 0.f), part[3]);
+            part[0] = fmaf(w4.x, fmaxf(__uint_as_float(r0[4 * h4 + 0]), 0.f), part[0]);
+            part[1] = fmaf(w4.y, fmaxf(__uint_as_float(r0[4 * h4 + 1]), 0.f), part[1]);
+            part[2] = fmaf(w4.z, fmaxf(__uint_as_float(r0[4 * h4 + 2]), 0.f), part[2]);
+            part[3] = fmaf(w4.w, fmaxf(__uint_as_float(r0[4 * h4 + 3]), 0.f), part[3]);
+          }
+#pragma unroll
+          for (int h4 = 0; h4 < 8; ++h4) {
+            const float4 w4 = wv[8 + h4];
+            part[0] = fmaf(w4.x, fmaxf(__uint_as_float(r1[4 * h4 + 0]), 0.f), part[0]);
+            part[1] = fmaf(w4.y, fmaxf(__uint_as_float(r1[4 * h4 + 1]), 0.f), part[1]);
+            part[2] = fmaf(w4.z, fmaxf(__uint_as_float(r1[4 * h4 + 2]), 0.f), part[2]);
+            part[3] = fmaf(w4.w, fmaxf(__uint_as_float(r1[4 * h4 + 3]), 0.f), part[3]);
           }
         }
         const float sc = ((part[0] + part[1]) + (part[2] + part[3])) * ks;
+        const bool visible = key < vis[j];
         if constexpr (FUSED) {
-          sc_s[j * p.chunk_cap + t * kTileKeys + kl] = key < vis[j] ? order_key(sc) : 0u;
+          const uint32_t u = order_key(sc);
+          sc_s[j * p.chunk_cap + t * kTileKeys + kl] = visible ? u : 0u;
+          if (visible) atomicAdd(&hist1[j * kHistBins + (u >> 21)], 1u);
         } else {
-          if (exists[j] && key < p.ld && t * kTileKeys + kl < chunk) {
-            p.scores[(static_cast<int64_t>(b) * p.n + row0 + j) * p.ld + key] = key < vis[j] ? sc : -INFINITY;
+          if (exists[j] && key < p.ld) {
+            p.scores[(static_cast<int64_t>(b) * p.n + row0 + j) * p.ld + key] = visible ? sc : -INFINITY;
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[a]);
+      if (lane == 0) {
+        mbar_arrive(&acc_empty[a]);
+        mbar_arrive(&empty[s]);
+      }
     }
   }
   __syncthreads();
+  if (trace && threadIdx.x == 0) tr[3] = globaltimer_ns();
 
   if constexpr (!FUSED) {
     // columns of this CTA's share that no tile covered: −inf
@@ -267,18 +330,24 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>::kT
     }
   } else {
     // agree across the cluster on whether anybody gave up
-    cluster_sync();
-    if (threadIdx.x == 0) {
-      int any = 0;
-      for (int r = 0; r < G; ++r) any |= static_cast<int>(dsmem_ld_u32(dsmem_addr((const void*)abort_flag, r)));
-      sel.any_abort = any;
+    if (G > 1) {
+      cluster_sync();
+      if (threadIdx.x == 0) {
+        int any = 0;
+        for (int r = 0; r < G; ++r) any |= static_cast<int>(dsmem_ld_u32(dsmem_addr((const void*)abort_flag, r)));
+        sel.any_abort = any;
+      }
+      __syncthreads();
+    } else {
+      if (threadIdx.x == 0) sel.any_abort = *abort_flag;
+      __syncthreads();
     }
-    __syncthreads();
     const bool skip = sel.any_abort != 0;
-    cluster_sync();
+    if (G > 1) cluster_sync();
 #pragma unroll 1
     for (int j = 0; j < NT; ++j) {
       if (!exists[j]) continue;
+      __syncthreads();   // the previous row's staged output has been written out
       int32_t* out = p.indices + (static_cast<int64_t>(b) * p.n + row0 + j) * p.k;
       const int v = vis[j];
       const int kt = min(p.k, v);
@@ -290,14 +359,16 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>::kT
         if (rank == 0)
           for (int i = (skip ? 0 : kt) + threadIdx.x; i < p.k; i += blockDim.x) out[i] = -1;
       } else {
-        cluster_select_row(sel, sc_s + j * p.chunk_cap, nloc, start, kt, out, G, rank);
+        cluster_select_row(sel, sc_s + j * p.chunk_cap, nloc, start, kt, hist1 + j * kHistBins, cand, C::kCand,
+                           out, G, rank, (trace && j == 0) ? tr : nullptr);
         if (rank == 0)
           for (int i = kt + threadIdx.x; i < p.k; i += blockDim.x) out[i] = -1;
       }
     }
-    cluster_sync();
+    if (G > 1) cluster_sync(); else __syncthreads();
   }
 
+  if (trace && threadIdx.x == 0) tr[4] = globaltimer_ns();
   // ------------------------------------------------------------ teardown
   if (warp == 0 && lane == 0) {
     // wait for copies still in flight (bounded) before the CTA's shared memory is released
@@ -314,6 +385,7 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>::kT
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+  if (trace && threadIdx.x == 0) tr[5] = globaltimer_ns();
 }
 
 // ---------------------------------------------------------------- host side
@@ -330,11 +402,11 @@ int pow2_floor(int x) {
   return p;
 }
 
-template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS>
+template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT>
 int launch_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
                  const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, float* scores,
                  int64_t ld, int k, int32_t* indices, cudaStream_t stream, int score_budget_bytes) {
-  using C = Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>;
+  using C = Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT>;
   const int ntb = (n + NT - 1) / NT;
   const int64_t items = static_cast<int64_t>(B) * ntb;
   const int sms = num_sms();
@@ -357,13 +429,15 @@ int launch_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, c
   if (smem > max_dynamic_smem()) return IDX_ERR_SHAPE;
   if (items * G > 0x7FFFFFFF) return IDX_ERR_SHAPE;
 
-  CUtensorMap tk, tq;
+  CUtensorMap tk, tq, ts;
   if (!make_tmap_u8_3d(&tk, k_cache, IDX_DIM, static_cast<uint64_t>(T_cap), static_cast<uint64_t>(B), kTileKeys))
     return IDX_ERR_ALIGN;
   if (!make_tmap_u8_3d(&tq, q_fp8, IDX_DIM, static_cast<uint64_t>(n) * IDX_HEADS, static_cast<uint64_t>(B), C::N))
     return IDX_ERR_ALIGN;
+  if (!make_tmap_f32_2d(&ts, k_scale_cache, static_cast<uint64_t>(T_cap), static_cast<uint64_t>(B), kTileKeys))
+    return IDX_ERR_ALIGN;
 
-  auto kern = score_kernel<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS>;
+  auto kern = score_kernel<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT>;
   static int configured_smem = -1;   // per instantiation
   if (configured_smem < smem) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -404,7 +478,7 @@ int launch_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, c
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, tk, tq, p) != cudaSuccess) return check_launch();
+  if (cudaLaunchKernelEx(&cfg, kern, tk, tq, ts, p) != cudaSuccess) return check_launch();
   return check_launch();
 }
 
@@ -415,7 +489,10 @@ int check_score_args(const uint8_t* q_fp8, const float* w, const uint8_t* k_cach
   if (!q_fp8 || !w || !k_cache || !k_scale_cache || !lengths) return IDX_ERR_NULL;
   if (max_len < n || max_len > T_cap || max_len > IDX_MAX_LEN) return IDX_ERR_SHAPE;
   if (causal != 0 && causal != 1) return IDX_ERR_SHAPE;
-  if ((reinterpret_cast<uintptr_t>(q_fp8) | reinterpret_cast<uintptr_t>(k_cache)) & 15) return IDX_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(q_fp8) | reinterpret_cast<uintptr_t>(k_cache) |
+       reinterpret_cast<uintptr_t>(k_scale_cache)) & 15)
+    return IDX_ERR_ALIGN;
+  if (T_cap % 4 != 0) return IDX_ERR_SHAPE;   // the scale rows are read by TMA: 16-byte pitch
   if (static_cast<int64_t>(n) * IDX_HEADS > 0x7FFFFFFF) return IDX_ERR_SHAPE;
   return 1;  // proceed
 }
@@ -439,9 +516,9 @@ extern "C" int idx_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_
   if (ld <= 0) return IDX_ERR_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (n <= kDecodeRowsMax)
-    return launch_score<1, false, 8, 4, 4>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
+    return launch_score<1, false, 6, 4, 8, 2>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
                                            scores, ld, 0, nullptr, s, 0);
-  return launch_score<4, false, 4, 2, 8>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
+  return launch_score<4, false, 4, 2, 8, 1>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
                                          scores, ld, 0, nullptr, s, 0);
 }
 
@@ -457,8 +534,24 @@ extern "C" int idx_score_topk(const uint8_t* q_fp8, const float* w, const uint8_
   if (!indices) return IDX_ERR_NULL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (n <= kDecodeRowsMax)
-    return launch_score<1, true, 8, 4, 4>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
+    return launch_score<1, true, 6, 4, 8, 2>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
                                           nullptr, 0, k, indices, s, 64 * 1024);
-  return launch_score<4, true, 4, 2, 8>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
+  return launch_score<4, true, 4, 2, 8, 1>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
                                         nullptr, 0, k, indices, s, 64 * 1024);
 }
+
+extern "C" int idx_debug_trace(unsigned long long* host_out, int max_ctas) {
+  if (!host_out || max_ctas <= 0) return IDX_ERR_NULL;
+  const int n = max_ctas < kTraceCtas ? max_ctas : kTraceCtas;
+  if (cudaMemcpyFromSymbol(host_out, g_trace, sizeof(unsigned long long) * kTraceSlots * n) != cudaSuccess)
+    return check_launch();
+  return IDX_OK;
+}
+
+namespace idx {
+unsigned long long* trace_buffer() {
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_trace) != cudaSuccess) return nullptr;
+  return static_cast<unsigned long long*>(ptr);
+}
+}  // namespace idx

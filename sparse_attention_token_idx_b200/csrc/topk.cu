@@ -16,6 +16,9 @@ namespace idx {
 namespace {
 
 constexpr int kTopkThreads = 256;
+constexpr int kTopkCand = 4096;   // candidate list entries
+
+constexpr int kTraceSlotsT = 16;
 
 struct TopkParams {
   const float* scores;
@@ -24,13 +27,18 @@ struct TopkParams {
   int64_t ld;
   int B, n, max_len, causal, k, G, chunk_cap;
   unsigned int* err;
+  unsigned long long* trace;   // per-CTA phase stamps, or null
 };
 
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);   // shared-space pointer
   SelectSmem& sel = *reinterpret_cast<SelectSmem*>(smem);
-  uint32_t* sc_s = reinterpret_cast<uint32_t*>(smem + sizeof(SelectSmem));
+  uint32_t* hist1 = reinterpret_cast<uint32_t*>(smem + sizeof(SelectSmem));
+  int* cand = reinterpret_cast<int*>(smem + sizeof(SelectSmem) + kHistBins * 4);
+  uint32_t* sc_s = reinterpret_cast<uint32_t*>(smem + sizeof(SelectSmem) + kHistBins * 4 + kTopkCand * 4);
+  unsigned long long* tr = (p.trace && blockIdx.x < 8192) ? p.trace + blockIdx.x * kTraceSlotsT : nullptr;
+  if (tr && threadIdx.x == 0) tr[0] = globaltimer_ns();
   const uint32_t rank = cluster_rank();
   const int G = p.G;
   const int64_t row = blockIdx.x / G;          // b * n + i
@@ -44,18 +52,40 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   const int start = static_cast<int>(rank) * chunk;
   const int nloc = max(0, min(start + chunk, vis) - start);
   const float* src = p.scores + row * p.ld + start;
-  for (int t = threadIdx.x; t < nloc; t += blockDim.x) sc_s[t] = order_key(__ldg(src + t));
+  for (int t = threadIdx.x; t < kHistBins; t += blockDim.x) hist1[t] = 0;
   __syncthreads();
+  // four independent loads in flight per thread
+  const int nthr = blockDim.x;
+  for (int t0 = threadIdx.x; t0 < nloc; t0 += 4 * nthr) {
+    float f[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int t = t0 + e * nthr;
+      f[e] = t < nloc ? __ldg(src + t) : 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int t = t0 + e * nthr;
+      if (t < nloc) {
+        const uint32_t u = order_key(f[e]);
+        sc_s[t] = u;
+        atomicAdd(&hist1[u >> 21], 1u);
+      }
+    }
+  }
+  __syncthreads();
+  if (tr && threadIdx.x == 0) tr[3] = globaltimer_ns();
   int32_t* out = p.indices + row * p.k;
   const int kt = min(p.k, vis);
   if (kt == vis) {
     for (int t = threadIdx.x; t < nloc; t += blockDim.x) out[start + t] = start + t;
   } else {
-    cluster_select_row(sel, sc_s, nloc, start, kt, out, G, rank);
+    cluster_select_row(sel, sc_s, nloc, start, kt, hist1, cand, kTopkCand, out, G, rank, tr);
   }
   if (rank == 0)
     for (int t = kt + threadIdx.x; t < p.k; t += blockDim.x) out[t] = -1;
-  cluster_sync();
+  if (G > 1) cluster_sync();
+  if (tr && threadIdx.x == 0) tr[4] = globaltimer_ns();
 }
 
 int pow2_floor_i(int x) {
@@ -86,8 +116,8 @@ extern "C" int idx_topk(const float* scores, const int32_t* lengths, int B, int 
   while (G > 1 && (max_len + G - 1) / G < 512) G /= 2;
   const int budget = 64 * 1024;
   while (G < 8 && static_cast<int64_t>((max_len + G - 1) / G) * 4 > budget) G *= 2;
-  const int chunk_cap = (max_len + G - 1) / G;
-  const int smem = 128 + static_cast<int>(sizeof(SelectSmem)) + chunk_cap * 4;
+  const int chunk_cap = ((max_len + G - 1) / G + 3) / 4 * 4;   // whole 16-byte vectors
+  const int smem = 128 + static_cast<int>(sizeof(SelectSmem)) + (kHistBins + kTopkCand) * 4 + chunk_cap * 4;
   if (smem > max_dynamic_smem()) return IDX_ERR_SHAPE;
   if (rows * G > 0x7FFFFFFF) return IDX_ERR_SHAPE;
   static int configured = -1;
@@ -96,7 +126,8 @@ extern "C" int idx_topk(const float* scores, const int32_t* lengths, int B, int 
       return check_launch();
     configured = smem;
   }
-  TopkParams p{scores, lengths, indices, ld, B, n, max_len, causal, k, G, chunk_cap, device_error_word()};
+  TopkParams p{scores, lengths, indices, ld, B, n, max_len, causal, k, G, chunk_cap, device_error_word(),
+               (debug_state().flags & 2u) ? trace_buffer() : nullptr};
   if (!p.err) return check_launch();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(rows * G), 1, 1);

@@ -45,8 +45,8 @@ class Case:
 
 def _to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """fp32 → bf16 bits, nearest-even (finite inputs)."""
-    u = np.ascontiguousarray(x, np.float32).view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    u = np.ascontiguousarray(x, np.float32).view(np.uint32)
+    u = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
     return u.astype(np.uint16)
 
 
