@@ -184,24 +184,25 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     keys, flops, key_rows, score_bytes = workload_numbers(case)
 
-    def step(ev=None):
-        ix.append(k_new, positions)
-        X.quant_queries(q, w_raw, case.fmt, q_out=q_fp8, w_out=w)
-        if ev is not None:
-            ev[0].record(stream)
+    # the kernel the roofline is about, timed on its own stream with events
+    def score_only():
         X.score_topk(q_fp8, w, ix.k_cache, ix.k_scale_cache, lengths, case.causal, case.k, max_len, out=out)
-        if ev is not None:
-            ev[1].record(stream)
 
+    graph, g_out = ix.capture(k_new, q, w_raw, positions, lengths, causal=case.causal, max_len=max_len)
+
+    def step():
+        graph.replay()
+
+    X.quant_queries_append(q, w_raw, k_new, positions, ix.k_cache, ix.k_scale_cache, case.fmt, q_fp8, w)
     for _ in range(args.warmup):
         step()
+        score_only()
     torch.cuda.synchronize()
     code, bits = X.status()
     if code != 0:
         raise RuntimeError(f"device error during warm-up: status {code}, bits {bits}")
 
-    # -------------------------------------------------------------- timed region
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # -------------------------------------------------------------- timed region: whole steps
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -210,13 +211,21 @@ def run_ours(args, rank, world, local_rank):
     with sampler:
         t0.record(stream)
         for i in range(args.steps):
-            step(evs[i])
+            step()
         t1.record(stream)
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     ms = t0.elapsed_time(t1)
-    score_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    # the fused score + top-k kernel alone, launch by launch on the same stream
+    n_k = min(args.steps, 500)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_k)]
+    for i in range(n_k):
+        evs[i][0].record(stream)
+        score_only()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    score_ms = sum(a.elapsed_time(b) for a, b in evs) / n_k
     code, bits = X.status()
     if code != 0:
         raise RuntimeError(f"device error in the timed region: status {code}, bits {bits}")
@@ -239,9 +248,12 @@ def run_ours(args, rank, world, local_rank):
         d_w.copy_(h_w, non_blocking=True)
         d_p.copy_(h_p, non_blocking=True)
         d_l.copy_(h_l, non_blocking=True)
-        idx = ix.step(d_k, d_q, d_w, d_p, d_l, causal=case.causal, max_len=max_len)
-        h_out.copy_(idx, non_blocking=True)
+        e2e_graph.replay()
+        h_out.copy_(e2e_out, non_blocking=True)
 
+    for d_t, h_t in ((d_k, h_k), (d_q, h_q), (d_w, h_w), (d_p, h_p), (d_l, h_l)):
+        d_t.copy_(h_t)
+    e2e_graph, e2e_out = ix.capture(d_k, d_q, d_w, d_p, d_l, causal=case.causal, max_len=max_len)
     e2e_steps = max(3, min(args.steps, 2000))
     for _ in range(args.warmup):
         step_e2e()
@@ -266,7 +278,7 @@ def run_ours(args, rank, world, local_rank):
     ms, score_ms, e2e_ms = t.tolist()
     return dict(case=case, keys=keys, flops=flops, key_rows=key_rows, score_bytes=score_bytes, ms=ms,
                 score_ms=score_ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
-                clocks=sampler.summary(), launches=3 * args.steps)
+                clocks=sampler.summary(), launches=2 * args.steps)
 
 
 def case_pinned(torch, a):

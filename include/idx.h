@@ -82,7 +82,7 @@ enum idx_status_code {
  *   x_bf16  [rows, 128]  bf16 input rows.
  *   x_fp8   [rows, 128]  out: e4m3 codes of fl32(y / scale), y = bf16(H·x/√128).
  *   x_scale [rows]       out: float32 scale per row.
- * rows may be 0 (nothing is enqueued).  x_bf16 and x_fp8 must be 8-byte aligned.
+ * rows may be 0 (nothing is enqueued).  x_bf16 and x_fp8 must be 16-byte aligned.
  */
 IDX_API int idx_quant(const uint16_t* x_bf16, int64_t rows, uint8_t* x_fp8, float* x_scale, int fmt,
               idx_stream_t stream);
@@ -95,6 +95,7 @@ IDX_API int idx_quant(const uint16_t* x_bf16, int64_t rows, uint8_t* x_fp8, floa
  *   q_bf16 [tokens, 64, 128], w_raw [tokens, 64] float32 in;
  *   q_fp8 [tokens, 64, 128] out; w [tokens, 64] float32 out (the folded weights
  *   idx_score / idx_score_topk take).  The query scales are not stored.
+ *   q_bf16 and q_fp8 must be 16-byte aligned.
  */
 IDX_API int idx_quant_queries(const uint16_t* q_bf16, const float* w_raw, int64_t tokens, uint8_t* q_fp8, float* w,
                       int fmt, idx_stream_t stream);
@@ -107,10 +108,21 @@ IDX_API int idx_quant_queries(const uint16_t* q_bf16, const float* w_raw, int64_
  *   k_cache       [B, T_cap, 128] uint8 (e4m3), written in place.
  *   k_scale_cache [B, T_cap] float32, written in place.
  * A sequence with positions[b] < 0 or positions[b] + n > T_cap is skipped and
- * IDX_DEV_ERR_POSITION is raised.
+ * IDX_DEV_ERR_POSITION is raised.  k_bf16 and k_cache must be 16-byte aligned.
  */
 IDX_API int idx_quant_append(const uint16_t* k_bf16, const int32_t* positions, int B, int n, uint8_t* k_cache,
                      float* k_scale_cache, int T_cap, int fmt, idx_stream_t stream);
+
+/*
+ * idx_quant_queries_append — idx_quant_queries and idx_quant_append of one
+ * indexer call in a single launch (the two are independent row sets of the
+ * same rotation + quantisation).  Arguments as in the two calls; either part
+ * may be empty (tokens = 0, or B = 0 / n = 0).
+ */
+IDX_API int idx_quant_queries_append(const uint16_t* q_bf16, const float* w_raw, int64_t tokens, uint8_t* q_fp8,
+                                     float* w, const uint16_t* k_bf16, const int32_t* positions, int B, int n,
+                                     uint8_t* k_cache, float* k_scale_cache, int T_cap, int fmt,
+                                     idx_stream_t stream);
 
 /*
  * idx_score — "Index scores" page: score equation and fp8_index docstring

@@ -34,6 +34,7 @@ SIGNATURES = {
     "idx_quant": (_I, [_P, _I64, _P, _P, _I, _P]),
     "idx_quant_queries": (_I, [_P, _P, _I64, _P, _P, _I, _P]),
     "idx_quant_append": (_I, [_P, _P, _I, _I, _P, _P, _I, _I, _P]),
+    "idx_quant_queries_append": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _I, _P, _P, _I, _I, _P]),
     "idx_score": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P]),
     "idx_topk": (_I, [_P, _P, _I, _I, _I64, _I, _I, _I, _P, _P, _SZ, _P]),
     "idx_score_topk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
@@ -127,6 +128,18 @@ def quant_append(k_new: torch.Tensor, positions: torch.Tensor, k_cache: torch.Te
                                    _ptr(k_cache, torch.uint8, "k_cache"),
                                    _ptr(k_scale_cache, torch.float32, "k_scale_cache"), T_cap, fmt,
                                    _stream(stream)), "idx_quant_append")
+
+
+def quant_queries_append(q, w_raw, k_new, positions, k_cache, k_scale_cache, fmt, q_out, w_out, stream=None):
+    """One launch: queries → (codes, folded weights) and new keys → cache slots."""
+    tokens = q.numel() // (HEADS * DIM)
+    B, n = k_new.shape[0], k_new.shape[1]
+    _check(load().idx_quant_queries_append(
+        _ptr(q, _BF16, "q"), _ptr(w_raw, torch.float32, "w_raw"), tokens, _ptr(q_out, torch.uint8, "q_out"),
+        _ptr(w_out, torch.float32, "w_out"), _ptr(k_new, _BF16, "k_new"), _ptr(positions, torch.int32, "positions"),
+        B, n, _ptr(k_cache, torch.uint8, "k_cache"), _ptr(k_scale_cache, torch.float32, "k_scale_cache"),
+        k_cache.shape[1], fmt, _stream(stream)), "idx_quant_queries_append")
+    return q_out, w_out
 
 
 def score(q_fp8, w, k_cache, k_scale_cache, lengths, causal: bool, max_len: int, ld: int | None = None,

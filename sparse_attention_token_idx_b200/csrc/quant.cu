@@ -1,14 +1,15 @@
 // Rotation + block-FP8 quantisation of 128-feature rows, and the key-cache
 // append ("Hadamard rotation" and "Index key cache" pages).
 //
-// One warp per row: lane l holds features 4l … 4l+3.  The Sylvester Hadamard
-// transform H_128 is seven butterfly stages in float64 (strides 1 and 2 inside
-// a lane, strides 4 … 64 across lanes with xor-shuffles), then one float64
-// multiply by the correctly rounded 128^-1/2 and one round-to-nearest-even to
-// bf16.  The quantiser takes amax over the 128 bf16 values (floored at 1e-4),
+// Four lanes per row: lane q holds features 32q … 32q+31.  The Sylvester
+// Hadamard transform H_128 is seven butterfly stages in float64 (strides 1 … 16
+// inside a lane, strides 32 and 64 across the four lanes with xor-shuffles),
+// then one float64 multiply by the correctly rounded 128^-1/2 and one
+// round-to-nearest-even to bf16.  The quantiser takes amax over the 128 bf16 values (floored at 1e-4),
 // scale = fl32(amax / 448) (IEEE division; ue8m0 rounds it up to a power of
 // two), and codes = e4m3(fl32(x / scale)) with the hardware's round-to-nearest-
-// even, saturating conversion.  Every warp stores one contiguous 128-byte row.
+// even, saturating conversion.  Each lane stores 32 contiguous code bytes.
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -22,30 +23,21 @@ namespace {
 constexpr unsigned long long kInvSqrtDBits = 0x3FB6A09E667F3BCDull;  // correctly rounded 2^-3.5 (binary64)
 constexpr uint32_t kInvSqrtDfBits = 0x3DB504F3u;                     // fl32(128^-1/2)
 constexpr uint32_t kAmaxFloorBits = 0x38D1B717u;                     // fl32(1e-4)
-constexpr int kRowsPerBlock = 8;                      // 8 warps
+constexpr int kWarpsPerBlock = 8;                     // 8 warps × 8 rows
 
 __device__ __forceinline__ float bf16_to_f32(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
-// float64 → bf16 bits, round to nearest even, from the binary64 / bfloat16
-// encodings: 8 significant bits, exponent range of binary32, subnormal quantum 2^-133.
-__device__ __forceinline__ uint32_t f64_to_bf16_rne(double v) {
-  const unsigned long long u = static_cast<unsigned long long>(__double_as_longlong(v));
-  const uint32_t sign = static_cast<uint32_t>(u >> 63) << 15;
-  const double a = fabs(v);
-  if (a < 0x1p-126) {
-    // subnormal (or zero) bf16: integer multiple of 2^-133, 128 · 2^-133 = smallest normal
-    const double m = rint(a * 0x1p133);  // exact scaling; rint rounds half to even
-    return sign | static_cast<uint32_t>(m);
-  }
-  unsigned long long mag = u & 0x7FFFFFFFFFFFFFFFull;
-  // keep 7 of the 52 fraction bits: add half-ulp minus one plus the kept LSB, truncate
-  mag += (1ull << 44) - 1 + ((mag >> 45) & 1ull);
-  mag &= ~((1ull << 45) - 1);
-  const int e64 = static_cast<int>(mag >> 52);           // biased binary64 exponent
-  const int e32 = e64 - 1023 + 127;                       // biased binary32/bf16 exponent
-  if (e32 >= 255) return sign | 0x7F80u;                  // overflow → inf
-  const uint32_t frac7 = static_cast<uint32_t>((mag >> 45) & 0x7Full);
-  return sign | (static_cast<uint32_t>(e32) << 7) | frac7;
+// float64 → bf16 value (as float), round to nearest even.  Two steps, from the
+// round-to-odd double-rounding property: rounding first to binary32 with "round
+// to odd" (truncate, then set the last bit if anything was lost) keeps enough
+// information that the hardware's round-to-nearest-even binary32 → bf16
+// conversion then gives the correctly rounded bf16 of the binary64 value
+// (binary32 carries 16 more significant bits than bf16, and reaches 2^-149 below
+// bf16's 2^-133 subnormal quantum).
+__device__ __forceinline__ float f64_to_bf16_as_f32(double v) {
+  float f = __double2float_rz(v);
+  if (static_cast<double>(f) != v) f = __uint_as_float(__float_as_uint(f) | 1u);
+  return __bfloat162float(__float2bfloat16_rn(f));
 }
 
 __device__ __forceinline__ float scale_from_amax(float amax, int fmt) {
@@ -63,83 +55,142 @@ __device__ __forceinline__ uint32_t e4m3x2(float hi, float lo) {
   return r;
 }
 
-// Rotate and quantise the row whose 4 features this lane holds (as bf16 bits).
-// Returns the lane's 4 codes packed little-endian and the row scale.
-__device__ __forceinline__ uint32_t rotate_quant_lane(uint2 in, int fmt, float* scale_out) {
-  const int lane = threadIdx.x & 31;
-  double v[4];
-  v[0] = bf16_to_f32(in.x & 0xFFFFu);
-  v[1] = bf16_to_f32(in.x >> 16);
-  v[2] = bf16_to_f32(in.y & 0xFFFFu);
-  v[3] = bf16_to_f32(in.y >> 16);
-  // stride 1: (0,1), (2,3)
-  double a0 = __dadd_rn(v[0], v[1]), a1 = __dsub_rn(v[0], v[1]);
-  double a2 = __dadd_rn(v[2], v[3]), a3 = __dsub_rn(v[2], v[3]);
-  // stride 2: (0,2), (1,3)
-  v[0] = __dadd_rn(a0, a2);
-  v[2] = __dsub_rn(a0, a2);
-  v[1] = __dadd_rn(a1, a3);
-  v[3] = __dsub_rn(a1, a3);
-  // strides 4 … 64: partner lane differs in bit m; the lower index keeps a+b, the upper a−b
+// Rows are handled by quads: 4 lanes per 128-feature row, lane q holding
+// features 32q … 32q+31, 8 rows per warp.  Strides 1 … 16 of the butterfly run
+// inside a lane; strides 32 and 64 pair lane q with q^1 and q^2.
+struct QuadRow {
+  uint4 codes[2];   // this lane's 32 e4m3 codes
+  float scale;
+};
+
+__device__ __forceinline__ QuadRow rotate_quant_quad(const uint4* src, int fmt) {
+  const int q = threadIdx.x & 3;
+  double v[32];
 #pragma unroll
-  for (int m = 1; m < 32; m <<= 1) {
-    const bool upper = (lane & m) != 0;
+  for (int i = 0; i < 4; ++i) {
+    const uint4 a = src[i];
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
+    for (int m = 0; m < 4; ++m) {
+      v[8 * i + 2 * m] = bf16_to_f32(w[m] & 0xFFFFu);
+      v[8 * i + 2 * m + 1] = bf16_to_f32(w[m] >> 16);
+    }
+  }
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if ((j & h) == 0) {
+        const double a = v[j], b = v[j + h];
+        v[j] = __dadd_rn(a, b);
+        v[j + h] = __dsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 1; m <= 2; m <<= 1) {
+    const bool upper = (q & m) != 0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
       const double o = __shfl_xor_sync(0xFFFFFFFFu, v[e], m);
       v[e] = upper ? __dsub_rn(o, v[e]) : __dadd_rn(v[e], o);
     }
   }
-  float x[4];
+  const double c = __longlong_as_double(static_cast<long long>(kInvSqrtDBits));
+  float x[32];
   float amax = 0.0f;
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    x[e] = bf16_to_f32(f64_to_bf16_rne(__dmul_rn(v[e], __longlong_as_double(static_cast<long long>(kInvSqrtDBits)))));
+  for (int e = 0; e < 32; ++e) {
+    x[e] = f64_to_bf16_as_f32(__dmul_rn(v[e], c));
     amax = fmaxf(amax, fabsf(x[e]));
   }
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+  QuadRow r;
+  r.scale = scale_from_amax(amax, fmt);
+  uint32_t pk[8];
 #pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, m));
-  const float s = scale_from_amax(amax, fmt);
-  *scale_out = s;
-  const uint32_t c01 = e4m3x2(__fdiv_rn(x[1], s), __fdiv_rn(x[0], s));
-  const uint32_t c23 = e4m3x2(__fdiv_rn(x[3], s), __fdiv_rn(x[2], s));
-  return c01 | (c23 << 16);
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t lo = e4m3x2(__fdiv_rn(x[4 * i + 1], r.scale), __fdiv_rn(x[4 * i], r.scale));
+    const uint32_t hi = e4m3x2(__fdiv_rn(x[4 * i + 3], r.scale), __fdiv_rn(x[4 * i + 2], r.scale));
+    pk[i] = lo | (hi << 16);
+  }
+  r.codes[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  r.codes[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  return r;
 }
 
-// MODE 0: plain rows.  MODE 1: query rows with weight folding.  MODE 2: cache append.
-template <int MODE>
-__global__ void __launch_bounds__(kRowsPerBlock * 32) quant_kernel(const uint16_t* __restrict__ x, int64_t rows,
-                                                                  uint8_t* __restrict__ codes,
-                                                                  float* __restrict__ scales, int fmt,
-                                                                  const float* __restrict__ w_raw,
-                                                                  float* __restrict__ w_out,
-                                                                  const int32_t* __restrict__ positions, int n,
-                                                                  int T_cap, unsigned int* err) {
+// One launch for any mix of:
+//   rows [0, plain_rows)              plain rows → codes / scales           (idx_quant)
+//   rows [0, q_rows)                  query rows → codes, folded weights    (idx_quant_queries)
+//   rows [q_rows, q_rows + k_rows)    key rows   → cache slots             (idx_quant_append)
+struct QuantArgs {
+  // plain / query rows
+  const uint16_t* x;
+  uint8_t* codes;
+  float* scales;          // plain rows only
+  const float* w_raw;     // query rows: fold weights when non-null
+  float* w_out;
+  int64_t rows;           // rows of the first kind
+  // key rows (append)
+  const uint16_t* k;
+  const int32_t* positions;
+  uint8_t* k_cache;
+  float* k_scale_cache;
+  int64_t k_rows;
+  int n, T_cap;
+  int fmt;
+  unsigned int* err;
+};
+
+__global__ void __launch_bounds__(kWarpsPerBlock * 32) quant_kernel(const QuantArgs a) {
   const int lane = threadIdx.x & 31;
-  const int64_t warps_total = static_cast<int64_t>(gridDim.x) * kRowsPerBlock;
-  for (int64_t r = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + (threadIdx.x >> 5); r < rows;
-       r += warps_total) {
-    int64_t dst_row = r;
-    if (MODE == 2) {
-      const int64_t b = r / n;
-      const int64_t i = r - b * n;
-      const int p = positions[b];
-      if (p < 0 || static_cast<int64_t>(p) + n > T_cap) {
-        if (lane == 0 && i == 0) raise_error(err, IDX_DEV_ERR_POSITION);
-        continue;
+  const int q = lane & 3;
+  const int64_t total = a.rows + a.k_rows;
+  const int64_t quads_total = static_cast<int64_t>(gridDim.x) * kWarpsPerBlock * 8;
+  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock + (threadIdx.x >> 5)) * 8; base < total;
+       base += quads_total) {
+    const int64_t r = base + (lane >> 2);
+    const bool live = r < total;
+    const bool is_key = live && r >= a.rows;
+    bool store = live;
+    const uint16_t* src;
+    uint8_t* dst;
+    int64_t slot = 0;
+    if (is_key) {
+      const int64_t kr = r - a.rows;
+      const int64_t b = kr / a.n;
+      const int64_t i = kr - b * a.n;
+      const int p = a.positions[b];
+      if (p < 0 || static_cast<int64_t>(p) + a.n > a.T_cap) {
+        if (q == 0 && i == 0) raise_error(a.err, IDX_DEV_ERR_POSITION);
+        store = false;
       }
-      dst_row = b * static_cast<int64_t>(T_cap) + p + i;
+      slot = b * static_cast<int64_t>(a.T_cap) + p + i;
+      src = a.k + kr * IDX_DIM;
+      dst = a.k_cache + slot * IDX_DIM;
+    } else if (live) {
+      src = a.x + r * IDX_DIM;
+      dst = a.codes + r * IDX_DIM;
+    } else {
+      // past the end: compute on a valid row (all lanes take part in the shuffles), store nothing
+      src = a.rows > 0 ? a.x : a.k;
+      dst = nullptr;
     }
-    const uint2 in = reinterpret_cast<const uint2*>(x + r * IDX_DIM)[lane];
-    float s;
-    const uint32_t packed = rotate_quant_lane(in, fmt, &s);
-    reinterpret_cast<uint32_t*>(codes + dst_row * IDX_DIM)[lane] = packed;
-    if (lane == 0) {
-      if (MODE == 1) {
-        const float w = __fmul_rn(__fmul_rn(__fmul_rn(w_raw[r], 0.125f), s), __uint_as_float(kInvSqrtDfBits));
-        w_out[r] = w;
-      } else {
-        scales[dst_row] = s;
+    const QuadRow out = rotate_quant_quad(reinterpret_cast<const uint4*>(src + 32 * q), a.fmt);
+    if (store) {
+      uint4* d = reinterpret_cast<uint4*>(dst + 32 * q);
+      d[0] = out.codes[0];
+      d[1] = out.codes[1];
+      if (q == 0) {
+        if (is_key) {
+          a.k_scale_cache[slot] = out.scale;
+        } else if (a.w_raw) {
+          a.w_out[r] = __fmul_rn(__fmul_rn(__fmul_rn(a.w_raw[r], 0.125f), out.scale),
+                                 __uint_as_float(kInvSqrtDfBits));
+        } else {
+          a.scales[r] = out.scale;
+        }
       }
     }
   }
@@ -153,9 +204,24 @@ __global__ void e4m3_encode_kernel(const float* __restrict__ x, int64_t count, u
 }
 
 int quant_grid(int64_t rows) {
-  const int64_t blocks = (rows + kRowsPerBlock - 1) / kRowsPerBlock;
-  const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
+  const int64_t rows_per_block = kWarpsPerBlock * 8;
+  const int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
   return static_cast<int>(blocks < cap ? blocks : cap);
+}
+
+int launch_quant(const QuantArgs& a, cudaStream_t stream) {
+  const int64_t total = a.rows + a.k_rows;
+  if (total == 0) return IDX_OK;
+  quant_kernel<<<quant_grid(total), kWarpsPerBlock * 32, 0, stream>>>(a);
+  return check_launch();
+}
+
+QuantArgs empty_args(int fmt) {
+  QuantArgs a = {};
+  a.fmt = fmt;
+  a.n = 1;
+  return a;
 }
 
 }  // namespace
@@ -170,37 +236,60 @@ extern "C" int idx_quant(const uint16_t* x_bf16, int64_t rows, uint8_t* x_fp8, f
   if (fmt != IDX_FMT_FP32 && fmt != IDX_FMT_UE8M0) return IDX_ERR_FMT;
   if (rows == 0) return IDX_OK;
   if (!x_bf16 || !x_fp8 || !x_scale) return IDX_ERR_NULL;
-  if ((reinterpret_cast<uintptr_t>(x_bf16) | reinterpret_cast<uintptr_t>(x_fp8)) & 7) return IDX_ERR_ALIGN;
-  quant_kernel<0><<<quant_grid(rows), kRowsPerBlock * 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      x_bf16, rows, x_fp8, x_scale, fmt, nullptr, nullptr, nullptr, 1, 0, nullptr);
-  return check_launch();
+  if ((reinterpret_cast<uintptr_t>(x_bf16) | reinterpret_cast<uintptr_t>(x_fp8)) & 15) return IDX_ERR_ALIGN;
+  QuantArgs a = empty_args(fmt);
+  a.x = x_bf16;
+  a.codes = x_fp8;
+  a.scales = x_scale;
+  a.rows = rows;
+  return launch_quant(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int idx_quant_queries(const uint16_t* q_bf16, const float* w_raw, int64_t tokens, uint8_t* q_fp8,
                                  float* w, int fmt, idx_stream_t stream) {
-  if (tokens < 0) return IDX_ERR_SHAPE;
-  if (fmt != IDX_FMT_FP32 && fmt != IDX_FMT_UE8M0) return IDX_ERR_FMT;
-  if (tokens == 0) return IDX_OK;
-  if (!q_bf16 || !w_raw || !q_fp8 || !w) return IDX_ERR_NULL;
-  if ((reinterpret_cast<uintptr_t>(q_bf16) | reinterpret_cast<uintptr_t>(q_fp8)) & 7) return IDX_ERR_ALIGN;
-  const int64_t rows = tokens * IDX_HEADS;
-  quant_kernel<1><<<quant_grid(rows), kRowsPerBlock * 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      q_bf16, rows, q_fp8, nullptr, fmt, w_raw, w, nullptr, 1, 0, nullptr);
-  return check_launch();
+  return idx_quant_queries_append(q_bf16, w_raw, tokens, q_fp8, w, nullptr, nullptr, 0, 0, nullptr, nullptr, 1, fmt,
+                                  stream);
 }
 
 extern "C" int idx_quant_append(const uint16_t* k_bf16, const int32_t* positions, int B, int n, uint8_t* k_cache,
                                 float* k_scale_cache, int T_cap, int fmt, idx_stream_t stream) {
-  if (B < 0 || n < 0 || T_cap <= 0) return IDX_ERR_SHAPE;
+  return idx_quant_queries_append(nullptr, nullptr, 0, nullptr, nullptr, k_bf16, positions, B, n, k_cache,
+                                  k_scale_cache, T_cap, fmt, stream);
+}
+
+extern "C" int idx_quant_queries_append(const uint16_t* q_bf16, const float* w_raw, int64_t tokens, uint8_t* q_fp8,
+                                        float* w, const uint16_t* k_bf16, const int32_t* positions, int B, int n,
+                                        uint8_t* k_cache, float* k_scale_cache, int T_cap, int fmt,
+                                        idx_stream_t stream) {
+  if (tokens < 0 || B < 0 || n < 0 || T_cap <= 0) return IDX_ERR_SHAPE;
   if (fmt != IDX_FMT_FP32 && fmt != IDX_FMT_UE8M0) return IDX_ERR_FMT;
-  if (B == 0 || n == 0) return IDX_OK;
-  if (n > T_cap) return IDX_ERR_SHAPE;
-  if (!k_bf16 || !positions || !k_cache || !k_scale_cache) return IDX_ERR_NULL;
-  if ((reinterpret_cast<uintptr_t>(k_bf16) | reinterpret_cast<uintptr_t>(k_cache)) & 7) return IDX_ERR_ALIGN;
-  const int64_t rows = static_cast<int64_t>(B) * n;
-  quant_kernel<2><<<quant_grid(rows), kRowsPerBlock * 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      k_bf16, rows, k_cache, k_scale_cache, fmt, nullptr, nullptr, positions, n, T_cap, device_error_word());
-  return check_launch();
+  const bool has_q = tokens > 0;
+  const bool has_k = B > 0 && n > 0;
+  if (has_k && n > T_cap) return IDX_ERR_SHAPE;
+  if (has_q && (!q_bf16 || !w_raw || !q_fp8 || !w)) return IDX_ERR_NULL;
+  if (has_k && (!k_bf16 || !positions || !k_cache || !k_scale_cache)) return IDX_ERR_NULL;
+  if (has_q && ((reinterpret_cast<uintptr_t>(q_bf16) | reinterpret_cast<uintptr_t>(q_fp8)) & 15)) return IDX_ERR_ALIGN;
+  if (has_k && ((reinterpret_cast<uintptr_t>(k_bf16) | reinterpret_cast<uintptr_t>(k_cache)) & 15)) return IDX_ERR_ALIGN;
+  QuantArgs a = empty_args(fmt);
+  if (has_q) {
+    a.x = q_bf16;
+    a.codes = q_fp8;
+    a.w_raw = w_raw;
+    a.w_out = w;
+    a.rows = tokens * IDX_HEADS;
+  }
+  if (has_k) {
+    a.k = k_bf16;
+    a.positions = positions;
+    a.k_cache = k_cache;
+    a.k_scale_cache = k_scale_cache;
+    a.k_rows = static_cast<int64_t>(B) * n;
+    a.n = n;
+    a.T_cap = T_cap;
+    a.err = device_error_word();
+    if (!a.err) return check_launch();
+  }
+  return launch_quant(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int idx_e4m3_encode(const float* x, int64_t count, uint8_t* out, idx_stream_t stream) {

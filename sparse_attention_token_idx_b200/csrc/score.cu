@@ -151,6 +151,11 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
   const int start = static_cast<int>(rank) * chunk;
   const int end = min(start + chunk, vis_max);
   const int ntiles = end > start ? ceil_div(end - start, kTileKeys) : 0;
+  // tile visiting order: rotated per work item so that CTAs do not walk
+  // equally-strided sequences in lockstep (tile t of the loop is tile rot(t))
+  const int rot = ((p.debug_flags & 4u) && ntiles > 0) ? (item * 37) % ntiles : 0;
+  auto tile_of = [&](int t) { const int u = t + rot; return u >= ntiles ? u - ntiles : u; };
+  const int pf_dist = (p.debug_flags & 8u) ? 8 : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -199,8 +204,10 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
         const int s = t % STAGES;
         if (!mbar_wait(&empty[s], ((t / STAGES) & 1) ^ 1, budget, abort_flag, p.err)) break;
         mbar_arrive_expect_tx(&full[s], kTileBytes + kTileKeys * 4);
-        tma_load_3d(k_s + s * kTileBytes, &tmap_k, &full[s], 0, start + t * kTileKeys, b);
-        tma_load_2d(scale_s + s * kTileKeys, &tmap_s, &full[s], start + t * kTileKeys, b);
+        const int tt = tile_of(t);
+        tma_load_3d(k_s + s * kTileBytes, &tmap_k, &full[s], 0, start + tt * kTileKeys, b);
+        tma_load_2d(scale_s + s * kTileKeys, &tmap_s, &full[s], start + tt * kTileKeys, b);
+        if (pf_dist && t + pf_dist < ntiles) tma_prefetch_3d(&tmap_k, 0, start + tile_of(t + pf_dist) * kTileKeys, b);
       }
       tma_issued = t;
     }
@@ -249,7 +256,8 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
     for (int t = tphase; t < ntiles; t += TSPLIT) {
       const int a = t % NUM_ACC;
       const int s = t % STAGES;
-      const int key = start + t * kTileKeys + kl;
+      const int tt = tile_of(t);
+      const int key = start + tt * kTileKeys + kl;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&acc_full[a], (t / NUM_ACC) & 1, budget, abort_flag, p.err) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -297,7 +305,7 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
         const bool visible = key < vis[j];
         if constexpr (FUSED) {
           const uint32_t u = order_key(sc);
-          sc_s[j * p.chunk_cap + t * kTileKeys + kl] = visible ? u : 0u;
+          sc_s[j * p.chunk_cap + tt * kTileKeys + kl] = visible ? u : 0u;
           if (visible) atomicAdd(&hist1[j * kHistBins + (u >> 21)], 1u);
         } else {
           if (exists[j] && key < p.ld) {
@@ -359,6 +367,10 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
         if (rank == 0)
           for (int i = (skip ? 0 : kt) + threadIdx.x; i < p.k; i += blockDim.x) out[i] = -1;
       } else {
+        if (p.debug_flags & 16u)   // experiment: run the selection twice (warm instruction cache)
+          cluster_select_row(sel, sc_s + j * p.chunk_cap, nloc, start, kt, hist1 + j * kHistBins, cand,
+                             C::kCand, out, G, rank, nullptr);
+        if (trace && j == 0 && threadIdx.x == 0) tr[6] = globaltimer_ns();
         cluster_select_row(sel, sc_s + j * p.chunk_cap, nloc, start, kt, hist1 + j * kHistBins, cand, C::kCand,
                            out, G, rank, (trace && j == 0) ? tr : nullptr);
         if (rank == 0)

@@ -34,12 +34,28 @@ class Indexer:
     def step(self, k_new, q, w_raw, positions, lengths, *, causal: bool, max_len: int, out=None, stream=None):
         """k_new [B, n, 128] bf16, q [B, n, 64, 128] bf16, w_raw [B, n, 64] fp32,
         positions [B] int32 (first new slot), lengths [B] int32 (= positions + n),
-        max_len ≥ max(lengths) on the host.  Returns top-k positions [B, n, k] int32."""
+        max_len ≥ max(lengths) on the host.  Returns top-k positions [B, n, k] int32.
+        Two launches: rotate + quantise queries and new keys (keys appended to the
+        cache), then the fused score + top-k."""
         B, n = q.shape[0], q.shape[1]
-        self.append(k_new, positions, stream=stream)
         q_fp8 = self._buf("q_fp8", tuple(q.shape), torch.uint8)
         w = self._buf("w", tuple(w_raw.shape), torch.float32)
-        X.quant_queries(q, w_raw, self.fmt, q_out=q_fp8, w_out=w, stream=stream)
+        X.quant_queries_append(q, w_raw, k_new, positions, self.k_cache, self.k_scale_cache, self.fmt, q_fp8, w,
+                               stream=stream)
         out = out if out is not None else self._buf("idx", (B, n, self.k), torch.int32)
         return X.score_topk(q_fp8, w, self.k_cache, self.k_scale_cache, lengths, causal, self.k, max_len,
                             out=out, stream=stream)
+
+    def capture(self, k_new, q, w_raw, positions, lengths, *, causal: bool, max_len: int):
+        """Record one step on static input tensors into a CUDA graph; returns
+        (graph, out) — replay the graph after refilling the inputs in place."""
+        out = self._buf("idx_graph", (q.shape[0], q.shape[1], self.k), torch.int32)
+        s = torch.cuda.Stream(device=self.device)
+        s.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(s):                      # warm-up outside the capture
+            self.step(k_new, q, w_raw, positions, lengths, causal=causal, max_len=max_len, out=out)
+        torch.cuda.current_stream(self.device).wait_stream(s)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.step(k_new, q, w_raw, positions, lengths, causal=causal, max_len=max_len, out=out)
+        return g, out
