@@ -155,6 +155,7 @@ def run_ours(args, rank, world, local_rank):
 
     from sparse_attention_token_idx_b200 import binding as X
     from sparse_attention_token_idx_b200 import synth
+    from sparse_attention_token_idx_b200.parallel import max_over_ranks
     from sparse_attention_token_idx_b200.pipeline import Indexer
 
     torch.cuda.set_device(local_rank)
@@ -272,10 +273,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device error in the end-to-end loop: status {code}, bits {bits}")
 
     # -------------------------------------------------------------- reduce over ranks (max time)
-    t = torch.tensor([ms, score_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, score_ms, e2e_ms = t.tolist()
+    ms, score_ms, e2e_ms = max_over_ranks([ms, score_ms, e2e_ms], device=dev)
     return dict(case=case, keys=keys, flops=flops, key_rows=key_rows, score_bytes=score_bytes, ms=ms,
                 score_ms=score_ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
                 clocks=sampler.summary(), launches=2 * args.steps)
