@@ -227,6 +227,21 @@ def run_ours(args, rank, world, local_rank):
         evs[i][1].record(stream)
     torch.cuda.synchronize()
     score_ms = sum(a.elapsed_time(b) for a, b in evs) / n_k
+    scoring_ms = None
+    if case.causal:
+        # prefill: the score contraction alone (unfused idx_score writing fp32 scores)
+        sc_buf = torch.empty((B, n, max_len), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            X.score(q_fp8, w, ix.k_cache, ix.k_scale_cache, lengths, case.causal, max_len, ld=max_len, out=sc_buf)
+        n_s = min(args.steps, 50)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(n_s):
+            X.score(q_fp8, w, ix.k_cache, ix.k_scale_cache, lengths, case.causal, max_len, ld=max_len, out=sc_buf)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        scoring_ms = s0.elapsed_time(s1) / n_s
+        del sc_buf
     code, bits = X.status()
     if code != 0:
         raise RuntimeError(f"device error in the timed region: status {code}, bits {bits}")
@@ -274,9 +289,11 @@ def run_ours(args, rank, world, local_rank):
 
     # -------------------------------------------------------------- reduce over ranks (max time)
     ms, score_ms, e2e_ms = max_over_ranks([ms, score_ms, e2e_ms], device=dev)
+    if scoring_ms is not None:
+        scoring_ms = max_over_ranks([scoring_ms], device=dev)[0]
     return dict(case=case, keys=keys, flops=flops, key_rows=key_rows, score_bytes=score_bytes, ms=ms,
                 score_ms=score_ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
-                clocks=sampler.summary(), launches=2 * args.steps)
+                clocks=sampler.summary(), launches=2 * args.steps, scoring_ms=scoring_ms)
 
 
 def case_pinned(torch, a):
@@ -443,6 +460,9 @@ def main():
     }
     if case.causal:
         line["tflops"] = r["flops"] * world / step_s / 1e12
+        sc_s = r["scoring_ms"] / 1e3
+        line["scoring"] = {"kernel": "idx_score (unfused, fp32 scores to HBM)", "us": r["scoring_ms"] * 1e3,
+                           "tflops": r["flops"] / sc_s / 1e12, "frac": r["flops"] / sc_s / 1e12 / (bf16 * FP8_PER_BF16)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case)
     if rank == 0:

@@ -137,16 +137,15 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
   const bool bad = len < p.n || len > p.max_len;
   if (bad && rank == 0 && threadIdx.x == 0) raise_error(p.err, IDX_DEV_ERR_LENGTH);
 
-  int vis[NT];
-  bool exists[NT];
+  // visible keys of row j of this block (0 for rows past n or a bad length)
+  auto row_exists = [&](int j) { return row0 + j < p.n; };
+  auto row_vis = [&](int j) {
+    const int tok = row0 + j;
+    return (tok < p.n && !bad) ? (p.causal ? len - p.n + tok + 1 : len) : 0;
+  };
   int vis_max = 0;
 #pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    const int tok = row0 + j;
-    exists[j] = tok < p.n;
-    vis[j] = (exists[j] && !bad) ? (p.causal ? len - p.n + tok + 1 : len) : 0;
-    vis_max = max(vis_max, vis[j]);
-  }
+  for (int j = 0; j < NT; ++j) vis_max = max(vis_max, row_vis(j));
   const int chunk = vis_max > 0 ? ceil_div(ceil_div(vis_max, G), kTileKeys) * kTileKeys : 0;
   const int start = static_cast<int>(rank) * chunk;
   const int end = min(start + chunk, vis_max);
@@ -248,10 +247,13 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
     const int tok_lo = ((ew >> 2) / TSPLIT) * C::kTokPerWarp;
     const int kl = quad * 32 + lane;            // key within the tile
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-    float wreg[C::kTokPerWarp == 1 ? 64 : 1];
+    // decode: this warp's 64 head weights in registers, packed in pairs for the
+    // f32x2 FMA; prefill (two rows per warp) reads them from shared memory
+    // (broadcast 16-byte loads) to stay within the register budget.
+    unsigned long long wp[C::kTokPerWarp == 1 ? 32 : 1];
     if constexpr (C::kTokPerWarp == 1) {
 #pragma unroll
-      for (int h = 0; h < 64; ++h) wreg[h] = w_s[tok_lo * 64 + h];
+      for (int i = 0; i < 32; ++i) wp[i] = pack2(w_s[tok_lo * 64 + 2 * i], w_s[tok_lo * 64 + 2 * i + 1]);
     }
     for (int t = tphase; t < ntiles; t += TSPLIT) {
       const int a = t % NUM_ACC;
@@ -268,47 +270,52 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
 #pragma unroll
       for (int jj = 0; jj < C::kTokPerWarp; ++jj) {
         const int j = tok_lo + jj;
-        uint32_t r0[32], r1[32];
-        tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64), r0);
-        tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64 + 32), r1);
-        tmem_wait();
-        tmem_regs_ready(r0);
-        tmem_regs_ready(r1);
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
+        unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
         if constexpr (C::kTokPerWarp == 1) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64), r0);
+          tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64 + 32), r1);
+          tmem_wait();
+          tmem_regs_ready(r0);
+          tmem_regs_ready(r1);
 #pragma unroll
-          for (int h = 0; h < 32; ++h)
-            part[h & 3] = fmaf(wreg[h], fmaxf(__uint_as_float(r0[h]), 0.f), part[h & 3]);
+          for (int i = 0; i < 16; ++i)
+            fma2(acc[i & 3], pack2(fmaxf(__uint_as_float(r0[2 * i]), 0.f), fmaxf(__uint_as_float(r0[2 * i + 1]), 0.f)),
+                 wp[i]);
 #pragma unroll
-          for (int h = 0; h < 32; ++h)
-            part[h & 3] = fmaf(wreg[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), part[h & 3]);
+          for (int i = 0; i < 16; ++i)
+            fma2(acc[i & 3], pack2(fmaxf(__uint_as_float(r1[2 * i]), 0.f), fmaxf(__uint_as_float(r1[2 * i + 1]), 0.f)),
+                 wp[16 + i]);
         } else {
-          const float4* wv = reinterpret_cast<const float4*>(w_s + j * 64);
 #pragma unroll
-          for (int h4 = 0; h4 < 8; ++h4) {
-            const float4 w4 = wv[h4];
-            part[0] = fmaf(w4.x, fmaxf(__uint_as_float(r0[4 * h4 + 0]), 0.f), part[0]);
-            part[1] = fmaf(w4.y, fmaxf(__uint_as_float(r0[4 * h4 + 1]), 0.f), part[1]);
-            part[2] = fmaf(w4.z, fmaxf(__uint_as_float(r0[4 * h4 + 2]), 0.f), part[2]);
-            part[3] = fmaf(w4.w, fmaxf(__uint_as_float(r0[4 * h4 + 3]), 0.f), part[3]);
-          }
+          for (int c = 0; c < 2; ++c) {
+            uint32_t r0[32];
+            tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64 + c * 32), r0);
+            tmem_wait();
+            tmem_regs_ready(r0);
+            const float4* wv = reinterpret_cast<const float4*>(w_s + j * 64 + c * 32);
 #pragma unroll
-          for (int h4 = 0; h4 < 8; ++h4) {
-            const float4 w4 = wv[8 + h4];
-            part[0] = fmaf(w4.x, fmaxf(__uint_as_float(r1[4 * h4 + 0]), 0.f), part[0]);
-            part[1] = fmaf(w4.y, fmaxf(__uint_as_float(r1[4 * h4 + 1]), 0.f), part[1]);
-            part[2] = fmaf(w4.z, fmaxf(__uint_as_float(r1[4 * h4 + 2]), 0.f), part[2]);
-            part[3] = fmaf(w4.w, fmaxf(__uint_as_float(r1[4 * h4 + 3]), 0.f), part[3]);
+            for (int i4 = 0; i4 < 8; ++i4) {
+              const float4 w4 = wv[i4];
+              fma2(acc[(2 * i4) & 3],
+                   pack2(fmaxf(__uint_as_float(r0[4 * i4]), 0.f), fmaxf(__uint_as_float(r0[4 * i4 + 1]), 0.f)),
+                   pack2(w4.x, w4.y));
+              fma2(acc[(2 * i4 + 1) & 3],
+                   pack2(fmaxf(__uint_as_float(r0[4 * i4 + 2]), 0.f), fmaxf(__uint_as_float(r0[4 * i4 + 3]), 0.f)),
+                   pack2(w4.z, w4.w));
+            }
           }
         }
+        const float2 p0 = unpack2(acc[0]), p1 = unpack2(acc[1]), p2 = unpack2(acc[2]), p3 = unpack2(acc[3]);
+        const float part[4] = {p0.x + p0.y, p1.x + p1.y, p2.x + p2.y, p3.x + p3.y};
         const float sc = ((part[0] + part[1]) + (part[2] + part[3])) * ks;
-        const bool visible = key < vis[j];
+        const bool visible = key < row_vis(j);
         if constexpr (FUSED) {
           const uint32_t u = order_key(sc);
           sc_s[j * p.chunk_cap + tt * kTileKeys + kl] = visible ? u : 0u;
           if (visible) atomicAdd(&hist1[j * kHistBins + (u >> 21)], 1u);
         } else {
-          if (exists[j] && key < p.ld) {
+          if (row_exists(j) && key < p.ld) {
             p.scores[(static_cast<int64_t>(b) * p.n + row0 + j) * p.ld + key] = visible ? sc : -INFINITY;
           }
         }
@@ -331,7 +338,7 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
     const int64_t lo = (vis_max == 0 && static_cast<int>(rank) == G - 1) ? 0 : col_lo;
     if (share_hi > lo) {
       for (int j = 0; j < NT; ++j) {
-        if (!exists[j]) continue;
+        if (!row_exists(j)) continue;
         float* row = p.scores + (static_cast<int64_t>(b) * p.n + row0 + j) * p.ld;
         for (int64_t c = lo + threadIdx.x; c < share_hi; c += blockDim.x) row[c] = -INFINITY;
       }
@@ -354,10 +361,10 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
     if (G > 1) cluster_sync();
 #pragma unroll 1
     for (int j = 0; j < NT; ++j) {
-      if (!exists[j]) continue;
+      if (!row_exists(j)) continue;
       __syncthreads();   // the previous row's staged output has been written out
       int32_t* out = p.indices + (static_cast<int64_t>(b) * p.n + row0 + j) * p.k;
-      const int v = vis[j];
+      const int v = row_vis(j);
       const int kt = min(p.k, v);
       const int nloc = max(0, min(end, v) - start);
       if (skip || kt == v) {
