@@ -232,11 +232,32 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Cluster barrier that orders only shared memory: each thread releases its
+// own prior shared::cta writes, arrives without further ordering, and after
+// the wait acquires shared::cluster data written by the other CTAs.  Much
+// cheaper than the release/acquire barrier when global stores are in flight.
+__device__ __forceinline__ void cluster_sync_shared() {
+  asm volatile(
+      "fence.release.sync_restrict::shared::cta.cluster;\n\t"
+      "barrier.cluster.arrive.relaxed.aligned;\n\t"
+      "barrier.cluster.wait.aligned;\n\t"
+      "fence.acquire.sync_restrict::shared::cluster.cluster;" ::: "memory");
+}
+
 // Address of the same shared variable in CTA `rank` of this cluster.
 __device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
   return r;
+}
+
+// Generic address of the same shared variable in CTA `rank` of this cluster:
+// plain (pipelinable, vectorisable) loads can then read it.
+template <typename T>
+__device__ __forceinline__ const T* dsmem_ptr(const T* local, uint32_t rank) {
+  uint64_t r;
+  asm volatile("mapa.u64 %0, %1, %2;" : "=l"(r) : "l"(reinterpret_cast<uint64_t>(local)), "r"(rank));
+  return reinterpret_cast<const T*>(r);
 }
 
 __device__ __forceinline__ uint32_t dsmem_ld_u32(uint32_t addr) {

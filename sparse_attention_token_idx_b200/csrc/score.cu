@@ -344,21 +344,9 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
       }
     }
   } else {
-    // agree across the cluster on whether anybody gave up
-    if (G > 1) {
-      cluster_sync();
-      if (threadIdx.x == 0) {
-        int any = 0;
-        for (int r = 0; r < G; ++r) any |= static_cast<int>(dsmem_ld_u32(dsmem_addr((const void*)abort_flag, r)));
-        sel.any_abort = any;
-      }
-      __syncthreads();
-    } else {
-      if (threadIdx.x == 0) sel.any_abort = *abort_flag;
-      __syncthreads();
-    }
-    const bool skip = sel.any_abort != 0;
-    if (G > 1) cluster_sync();
+    // Whether some CTA of the cluster gave up is learnt inside the selection
+    // (its first exchange); rows where every visible position is selected need
+    // no scores and are written regardless.
 #pragma unroll 1
     for (int j = 0; j < NT; ++j) {
       if (!row_exists(j)) continue;
@@ -367,19 +355,15 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
       const int v = row_vis(j);
       const int kt = min(p.k, v);
       const int nloc = max(0, min(end, v) - start);
-      if (skip || kt == v) {
-        // every visible position is selected (or the launch gave up): slot s holds position s
-        if (!skip)
-          for (int i = threadIdx.x; i < nloc; i += blockDim.x) out[start + i] = start + i;
+      if (kt == v) {
+        // every visible position is selected: slot s holds position s
+        for (int i = threadIdx.x; i < nloc; i += blockDim.x) out[start + i] = start + i;
         if (rank == 0)
-          for (int i = (skip ? 0 : kt) + threadIdx.x; i < p.k; i += blockDim.x) out[i] = -1;
+          for (int i = kt + threadIdx.x; i < p.k; i += blockDim.x) out[i] = -1;
       } else {
-        if (p.debug_flags & 16u)   // experiment: run the selection twice (warm instruction cache)
-          cluster_select_row(sel, sc_s + j * p.chunk_cap, nloc, start, kt, hist1 + j * kHistBins, cand,
-                             C::kCand, out, G, rank, nullptr);
         if (trace && j == 0 && threadIdx.x == 0) tr[6] = globaltimer_ns();
         cluster_select_row(sel, sc_s + j * p.chunk_cap, nloc, start, kt, hist1 + j * kHistBins, cand, C::kCand,
-                           out, G, rank, (trace && j == 0) ? tr : nullptr);
+                           out, G, rank, (trace && j == 0) ? tr : nullptr, const_cast<const int*>(abort_flag));
         if (rank == 0)
           for (int i = kt + threadIdx.x; i < p.k; i += blockDim.x) out[i] = -1;
       }
@@ -555,7 +539,7 @@ extern "C" int idx_score_topk(const uint8_t* q_fp8, const float* w, const uint8_
   if (n <= kDecodeRowsMax)
     return launch_score<1, true, 6, 4, 8, 2>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
                                           nullptr, 0, k, indices, s, 64 * 1024);
-  return launch_score<4, true, 4, 2, 8, 1>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
+  return launch_score<4, true, 3, 2, 8, 1>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
                                         nullptr, 0, k, indices, s, 64 * 1024);
 }
 

@@ -44,16 +44,17 @@ struct Grp {
 };
 
 struct SelectSmem {
-  uint32_t hist[kHistBins];      // this CTA's level-2/3 histogram
+  uint32_t hist[kHistBins];      // this CTA's level-2 histogram
+  uint32_t hist3[kHistBins / 2]; // this CTA's level-3 histogram (own buffer: one barrier per exchange)
   uint32_t hsum[kHistBins];      // cluster-summed histogram
   int warp_a[32];
   int warp_b[32];
   int bin;
   int above;
-  int cta_cnt[2];                // this CTA's totals of the current pass (read by the cluster)
+  int cta_cnt[2][2];             // this CTA's pass totals, double-buffered by exchange parity
   int cta_base[2];               // cluster prefix of those totals for this CTA
   int any_abort;
-  int pad[1];
+  int pad[3];
   int32_t out_s[kStage];         // staged positions of the current row (CTA 0's copy is the one used)
 };
 
@@ -104,6 +105,10 @@ __device__ __forceinline__ void find_bin(SelectSmem& sm, const uint32_t* hist, i
   const int lo = hi - per;
   int csum = 0;
   for (int bn = (lo > 0 ? lo : 0); bn < hi; ++bn) csum += static_cast<int>(hist[bn]);
+  if (tid == 0) {   // safe defaults should no bin hold the rem-th element (cannot happen on valid data)
+    sm.bin = 0;
+    sm.above = 0;
+  }
   int excl, dummy, tot, tot2;
   block_scan2(sm, csum, 0, excl, dummy, tot, tot2);
   if (csum > 0 && excl < rem && rem <= excl + csum) {
@@ -121,37 +126,56 @@ __device__ __forceinline__ void find_bin(SelectSmem& sm, const uint32_t* hist, i
   __syncthreads();
 }
 
-// Publish this CTA's pass totals (cta_cnt), then — between the two cluster
-// barriers — sum `local` (nb bins, may be 0) over the cluster into sm.hsum and
-// read the lower ranks' totals into sm.cta_base.  Entry: every CTA's `local`
-// and cta_cnt are final (the caller wrote cta_cnt before its last
-// __syncthreads).  Exit: hsum / cta_base ready; `local` may be reused.
+// Exchange over the cluster: after one barrier, sum `local` (nb bins) of all
+// CTAs into sm.hsum, or (nb = 0) read the lower ranks' pass totals
+// cta_cnt[parity] into sm.cta_base.  Entry: every CTA's `local` / cta_cnt are
+// final.  Each exchanged buffer is written again only after a later barrier,
+// which no CTA passes before finishing its reads here.
 template <bool CL>
 __device__ __forceinline__ void cluster_exchange(SelectSmem& sm, const uint32_t* local, int nb, int G,
-                                                 uint32_t rank) {
+                                                 uint32_t rank, int parity, const int* abort_flag = nullptr) {
   __syncthreads();
-  Grp<CL>::sync();
   if constexpr (CL) {
-    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
-      uint32_t v[8];
+    // One shared-memory barrier: every buffer read here is written again only
+    // after a later barrier, which no CTA passes before finishing these reads.
+    cluster_sync_shared();
+    // 16-byte loads from every rank's histogram through generic pointers, all
+    // independent, so that the remote reads overlap
+    const uint4* src[8];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) v[r] = r < G ? dsmem_ld_u32(dsmem_addr(&local[i], r)) : 0u;
-      uint32_t s = 0;
+    for (int r = 0; r < 8; ++r) src[r] = reinterpret_cast<const uint4*>(dsmem_ptr(local, r < G ? r : 0));
+    for (int i4 = threadIdx.x; i4 < nb / 4; i4 += blockDim.x) {
+      uint4 acc = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-      for (int r = 0; r < 8; ++r) s += v[r];
-      sm.hsum[i] = s;
+      for (int r = 0; r < 8; ++r) {
+        if (r < G) {
+          const uint4 v = src[r][i4];
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+      }
+      reinterpret_cast<uint4*>(sm.hsum)[i4] = acc;
     }
-    if (threadIdx.x < 2) {
+    if (nb == 0 && threadIdx.x < 2) {
       int base = 0;
       for (int r = 0; r < static_cast<int>(rank); ++r)
-        base += static_cast<int>(dsmem_ld_u32(dsmem_addr(&sm.cta_cnt[threadIdx.x], r)));
+        base += static_cast<int>(dsmem_ld_u32(dsmem_addr(&sm.cta_cnt[parity][threadIdx.x], r)));
       sm.cta_base[threadIdx.x] = base;
     }
+    if (abort_flag && threadIdx.x == 32) {
+      int any = 0;
+      for (int r = 0; r < G; ++r) any |= *dsmem_ptr(abort_flag, r);
+      sm.any_abort = any;
+    }
+    __syncthreads();
   } else {
     for (int i = threadIdx.x; i < nb; i += blockDim.x) sm.hsum[i] = local[i];
     if (threadIdx.x < 2) sm.cta_base[threadIdx.x] = 0;
+    if (abort_flag && threadIdx.x == 32) sm.any_abort = *abort_flag;
+    __syncthreads();
   }
-  Grp<CL>::sync();
 }
 
 // Output writer of one row: positions go to CTA 0's staging buffer when the row
@@ -173,21 +197,25 @@ struct RowOut {
   }
 };
 
-// End of a row: all staged positions are in CTA 0's buffer after the barrier;
-// CTA 0 writes them out with coalesced stores.  The barrier also lets the next
-// row reuse the exchange buffers.
+// End of a row: all staged positions are in CTA 0's buffer after the barrier
+// (a full release/acquire barrier: the staging stores went to another CTA's
+// shared memory); CTA 0 writes them out with coalesced stores.
 template <bool CL>
 __device__ __forceinline__ void flush_row(SelectSmem& sm, const RowOut<CL>& ro, int kt, uint32_t rank) {
   Grp<CL>::sync();
-  if (ro.staged && rank == 0)
-    for (int i = threadIdx.x; i < kt; i += blockDim.x) ro.out[i] = sm.out_s[i];
+  if (rank == 0) {
+    if (sm.any_abort)   // a CTA of the cluster gave up: its scores are not valid
+      for (int i = threadIdx.x; i < kt; i += blockDim.x) ro.out[i] = -1;
+    else if (ro.staged)
+      for (int i = threadIdx.x; i < kt; i += blockDim.x) ro.out[i] = sm.out_s[i];
+  }
 }
 
 // Exchange only the per-CTA pass totals (no histogram).
 template <bool CL>
-__device__ __forceinline__ void exchange_counts(SelectSmem& sm, int G, uint32_t rank) {
+__device__ __forceinline__ void exchange_counts(SelectSmem& sm, int G, uint32_t rank, int parity) {
   if constexpr (CL) {
-    cluster_exchange<true>(sm, nullptr, 0, G, rank);
+    cluster_exchange<true>(sm, nullptr, 0, G, rank, parity);
   } else {
     if (threadIdx.x < 2) sm.cta_base[threadIdx.x] = 0;
     __syncthreads();
@@ -198,11 +226,12 @@ __device__ __forceinline__ void exchange_counts(SelectSmem& sm, int G, uint32_t 
 // single CTA reads its own histogram in place.
 template <bool CL>
 __device__ __forceinline__ const uint32_t* summed_hist(SelectSmem& sm, const uint32_t* local, int nb, int G,
-                                                       uint32_t rank) {
+                                                       uint32_t rank, const int* abort_flag = nullptr) {
   if constexpr (CL) {
-    cluster_exchange<true>(sm, local, nb, G, rank);
+    cluster_exchange<true>(sm, local, nb, G, rank, 0, abort_flag);
     return sm.hsum;
   } else {
+    if (abort_flag && threadIdx.x == 0) sm.any_abort = *abort_flag;
     __syncthreads();
     return local;
   }
@@ -220,20 +249,26 @@ template <bool CL>
 __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint32_t* keys, int nloc, int start,
                                                      int kt, const uint32_t* hist1, int* cand, int cap,
                                                      int32_t* out, int G, uint32_t rank,
-                                                     unsigned long long* tr) {
+                                                     unsigned long long* tr, const int* abort_flag) {
   const int tid = threadIdx.x, nthr = blockDim.x;
   auto stamp = [&](int slot) {
     if (tr && tid == 0) tr[slot] = globaltimer_ns();
   };
+  if (tid == 0) sm.any_abort = 0;
   RowOut<CL> ro;
   ro.out = out;
   ro.staged = kt <= kStage;
   ro.stage_local = sm.out_s;
   ro.stage_base = CL ? dsmem_addr(sm.out_s, 0) : 0u;
   for (int i = tid; i < kHistBins; i += nthr) sm.hist[i] = 0;
+  for (int i = tid; i < kHistBins / 2; i += nthr) sm.hist3[i] = 0;
 
   // ---- level 1
-  const uint32_t* H = summed_hist<CL>(sm, hist1, kHistBins, G, rank);
+  const uint32_t* H = summed_hist<CL>(sm, hist1, kHistBins, G, rank, abort_flag);
+  if (sm.any_abort) {   // same value in every CTA of the cluster: skip the selection, flush writes -1
+    flush_row<CL>(sm, ro, kt, rank);
+    return;
+  }
   find_bin(sm, H, kHistBins, kt);
   const uint32_t b1 = static_cast<uint32_t>(sm.bin);
   int rem = kt - sm.above;
@@ -260,8 +295,8 @@ __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint3
   stamp(9);
   int og, oe, tg, te;
   block_scan2(sm, cg, ce, og, oe, tg, te);
-  if (tid == 0) sm.cta_cnt[0] = tg;
-  exchange_counts<CL>(sm, G, rank);
+  if (tid == 0) sm.cta_cnt[0][0] = tg;
+  exchange_counts<CL>(sm, G, rank, 0);
   const bool overflow = te > cap;
   stamp(10);
   if (tr && tid == 0) tr[15] = static_cast<unsigned long long>(te);
@@ -311,8 +346,6 @@ __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint3
   rem -= sm.above;
   const bool done2 = static_cast<int>(H2[b2]) == rem;
   __syncthreads();                           // everyone has read H2 (it may be sm.hist)
-  for (int i = tid; i < 1024; i += nthr) sm.hist[i] = 0;
-  __syncthreads();
   // ---- pass B: over the candidates
   const int trips_b = (nscan + nthr - 1) / nthr;
   cg = 0;
@@ -324,14 +357,14 @@ __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint3
         const uint32_t mid = (key >> 10) & 0x7FF;
         const bool eq = mid == b2;
         cg += (mid > b2 || (done2 && eq)) ? 1 : 0;
-        if (!done2 && eq) atomicAdd(&sm.hist[key & 0x3FF], 1u);
+        if (!done2 && eq) atomicAdd(&sm.hist3[key & 0x3FF], 1u);
       }
     }
   }
   stamp(12);
   block_scan2(sm, cg, 0, og, oe, tg, te);
-  if (tid == 0) sm.cta_cnt[0] = tg;
-  exchange_counts<CL>(sm, G, rank);
+  if (tid == 0) sm.cta_cnt[1][0] = tg;
+  exchange_counts<CL>(sm, G, rank, 1);
   {
     int wg = out_base + sm.cta_base[0] + og;
     for (int it = 0; it < trips_b; ++it) {
@@ -352,7 +385,7 @@ __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint3
   }
   stamp(13);
   // ---- level 3
-  const uint32_t* H3 = summed_hist<CL>(sm, sm.hist, 1024, G, rank);
+  const uint32_t* H3 = summed_hist<CL>(sm, sm.hist3, 1024, G, rank);
   find_bin(sm, H3, 1024, rem);
   const uint32_t b3 = static_cast<uint32_t>(sm.bin);
   const int above3 = sm.above;
@@ -375,10 +408,10 @@ __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint3
   }
   block_scan2(sm, cg, ce, og, oe, tg, te);
   if (tid == 0) {
-    sm.cta_cnt[0] = tg;
-    sm.cta_cnt[1] = te;
+    sm.cta_cnt[0][0] = tg;
+    sm.cta_cnt[0][1] = te;
   }
-  exchange_counts<CL>(sm, G, rank);
+  exchange_counts<CL>(sm, G, rank, 0);
   {
     int wg = n_gt - above3 + sm.cta_base[0] + og;
     int we = sm.cta_base[1] + oe;
@@ -406,11 +439,12 @@ __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint3
 __device__ __forceinline__ void cluster_select_row(SelectSmem& sm, const uint32_t* keys, int nloc, int start,
                                                    int kt, const uint32_t* hist1, int* cand, int cap,
                                                    int32_t* out, int G, uint32_t rank,
-                                                   unsigned long long* tr = nullptr) {
+                                                   unsigned long long* tr = nullptr,
+                                                   const int* abort_flag = nullptr) {
   if (G == 1)
-    cluster_select_row_t<false>(sm, keys, nloc, start, kt, hist1, cand, cap, out, G, rank, tr);
+    cluster_select_row_t<false>(sm, keys, nloc, start, kt, hist1, cand, cap, out, G, rank, tr, abort_flag);
   else
-    cluster_select_row_t<true>(sm, keys, nloc, start, kt, hist1, cand, cap, out, G, rank, tr);
+    cluster_select_row_t<true>(sm, keys, nloc, start, kt, hist1, cand, cap, out, G, rank, tr, abort_flag);
 }
 
 }  // namespace idx
