@@ -5,7 +5,7 @@
 // Hadamard transform H_128 is seven butterfly stages in float64 (strides 1 … 16
 // inside a lane, strides 32 and 64 across the four lanes with xor-shuffles),
 // then one float64 multiply by the correctly rounded 128^-1/2 and one
-// round-to-nearest-even to bf16.  The quantiser takes amax over the 128 bf16 values (floored at 1e-4),
+// round-to-nearest-even to bf16 (cvt.rn.bf16.f64).  The quantiser takes amax over the 128 bf16 values (floored at 1e-4),
 // scale = fl32(amax / 448) (IEEE division; ue8m0 rounds it up to a power of
 // two), and codes = e4m3(fl32(x / scale)) with the hardware's round-to-nearest-
 // even, saturating conversion.  Each lane stores 32 contiguous code bytes.
@@ -27,17 +27,12 @@ constexpr int kWarpsPerBlock = 8;                     // 8 warps × 8 rows
 
 __device__ __forceinline__ float bf16_to_f32(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
-// float64 → bf16 value (as float), round to nearest even.  Two steps, from the
-// round-to-odd double-rounding property: rounding first to binary32 with "round
-// to odd" (truncate, then set the last bit if anything was lost) keeps enough
-// information that the hardware's round-to-nearest-even binary32 → bf16
-// conversion then gives the correctly rounded bf16 of the binary64 value
-// (binary32 carries 16 more significant bits than bf16, and reaches 2^-149 below
-// bf16's 2^-133 subnormal quantum).
+// float64 → bf16 value (as float), round to nearest even (the PTX conversion
+// cvt.rn.bf16.f64 rounds the binary64 value once, subnormals included).
 __device__ __forceinline__ float f64_to_bf16_as_f32(double v) {
-  float f = __double2float_rz(v);
-  if (static_cast<double>(f) != v) f = __uint_as_float(__float_as_uint(f) | 1u);
-  return __bfloat162float(__float2bfloat16_rn(f));
+  uint16_t h;
+  asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(h) : "d"(v));
+  return __uint_as_float(static_cast<uint32_t>(h) << 16);
 }
 
 __device__ __forceinline__ float scale_from_amax(float amax, int fmt) {
@@ -54,6 +49,19 @@ __device__ __forceinline__ uint32_t e4m3x2(float hi, float lo) {
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
 }
+
+// x / s, correctly rounded (IEEE binary32 division), for the quantiser.
+// ue8m0 scales are powers of two, so x times the exact reciprocal is the same
+// value (one rounding of the same exact quotient); other scales divide.
+struct Divider {
+  float s, y;
+  bool pow2;
+  __device__ __forceinline__ Divider(float scale, int fmt) : s(scale) {
+    pow2 = fmt == IDX_FMT_UE8M0;
+    y = pow2 ? __frcp_rn(scale) : 0.f;
+  }
+  __device__ __forceinline__ float div(float x) const { return pow2 ? __fmul_rn(x, y) : __fdiv_rn(x, s); }
+};
 
 // Rows are handled by quads: 4 lanes per 128-feature row, lane q holding
 // features 32q … 32q+31, 8 rows per warp.  Strides 1 … 16 of the butterfly run
@@ -87,13 +95,16 @@ __device__ __forceinline__ QuadRow rotate_quant_quad(const uint4* src, int fmt) 
       }
     }
   }
+  // cross-lane stages: the lower index keeps a + b, the upper gets a − b, i.e.
+  // partner ± own — one FMA with ±1 (exact product, one rounding: the same
+  // value as the add or subtract)
 #pragma unroll
   for (int m = 1; m <= 2; m <<= 1) {
-    const bool upper = (q & m) != 0;
+    const double sgn = (q & m) ? -1.0 : 1.0;
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const double o = __shfl_xor_sync(0xFFFFFFFFu, v[e], m);
-      v[e] = upper ? __dsub_rn(o, v[e]) : __dadd_rn(v[e], o);
+      v[e] = __fma_rn(sgn, v[e], o);
     }
   }
   const double c = __longlong_as_double(static_cast<long long>(kInvSqrtDBits));
@@ -108,11 +119,12 @@ __device__ __forceinline__ QuadRow rotate_quant_quad(const uint4* src, int fmt) 
   amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
   QuadRow r;
   r.scale = scale_from_amax(amax, fmt);
+  const Divider dv(r.scale, fmt);
   uint32_t pk[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t lo = e4m3x2(__fdiv_rn(x[4 * i + 1], r.scale), __fdiv_rn(x[4 * i], r.scale));
-    const uint32_t hi = e4m3x2(__fdiv_rn(x[4 * i + 3], r.scale), __fdiv_rn(x[4 * i + 2], r.scale));
+    const uint32_t lo = e4m3x2(dv.div(x[4 * i + 1]), dv.div(x[4 * i]));
+    const uint32_t hi = e4m3x2(dv.div(x[4 * i + 3]), dv.div(x[4 * i + 2]));
     pk[i] = lo | (hi << 16);
   }
   r.codes[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);

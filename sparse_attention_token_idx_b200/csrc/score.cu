@@ -55,7 +55,7 @@ struct ScoreParams {
   unsigned int* err;         // device error word
 };
 
-template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT>
+template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT, bool W_REGS>
 struct Cfg {
   static constexpr int N = NT * IDX_HEADS;
   static constexpr int kThreads = (2 + EPI_WARPS) * 32;
@@ -89,11 +89,11 @@ struct Cfg {
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT>
-__global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT>::kThreads, 1)
+template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT, bool W_REGS>
+__global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>::kThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                  const __grid_constant__ CUtensorMap tmap_s, const ScoreParams p) {
-  using C = Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT>;
+  using C = Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>;
   constexpr int N = C::N;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base (128-byte swizzle atoms), kept as a shared-space pointer
@@ -150,12 +150,10 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
   const int start = static_cast<int>(rank) * chunk;
   const int end = min(start + chunk, vis_max);
   const int ntiles = end > start ? ceil_div(end - start, kTileKeys) : 0;
-  // tile visiting order: rotated per work item so that CTAs do not walk
-  // equally-strided sequences in lockstep (tile t of the loop is tile rot(t))
-  const int rot = ((p.debug_flags & 4u) && ntiles > 0) ? (item * 37) % ntiles : 0;
-  auto tile_of = [&](int t) { const int u = t + rot; return u >= ntiles ? u - ntiles : u; };
-  const int pf_dist = (p.debug_flags & 8u) ? 8 : 0;
+  auto tile_of = [](int t) { return t; };   // tiles are visited in order
 
+  int tma_issued = 0;     // producer lane (thread 0): K tiles whose loads were issued
+  bool q_issued = false;  // producer lane: the query load was issued
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -170,6 +168,25 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
     mbar_init(never_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
+    // Thread 0 is also the TMA producer: start the query and the first STAGES
+    // key tiles now, so that their DRAM latency overlaps the rest of the set-up
+    // (the ring is empty, no slot needs to be waited for).
+    if (ntiles > 0) {
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_q);
+      tma_prefetch_desc(&tmap_s);
+      mbar_arrive_expect_tx(q_full, C::kQBytes);
+      tma_load_3d(q_s, &tmap_q, q_full, 0, row0 * IDX_HEADS, b);
+      q_issued = true;
+      const int pre = ntiles < STAGES ? ntiles : STAGES;
+      for (int t = 0; t < pre; ++t) {
+        mbar_arrive_expect_tx(&full[t], kTileBytes + kTileKeys * 4);
+        const int tt = tile_of(t);
+        tma_load_3d(k_s + t * kTileBytes, &tmap_k, &full[t], 0, start + tt * kTileKeys, b);
+        tma_load_2d(scale_s + t * kTileKeys, &tmap_s, &full[t], start + tt * kTileKeys, b);
+      }
+      tma_issued = pre;
+    }
   }
   if (warp == 1) tmem_alloc(tmem_slot, C::kTmemCols);
   for (int i = threadIdx.x; i < N; i += blockDim.x) {
@@ -185,20 +202,12 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
   const uint32_t tmem_base = *tmem_slot;
   const uint64_t budget = p.budget_ns;
   if (trace && threadIdx.x == 0) tr[1] = globaltimer_ns();
-  int tma_issued = 0;   // producer lane: K tiles whose loads were issued
-  bool q_issued = false;  // producer lane: the query load was issued
   bool mma_issued = false;  // MMA lane: at least one tcgen05.mma issued
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && ntiles > 0) {
-      tma_prefetch_desc(&tmap_k);
-      tma_prefetch_desc(&tmap_q);
-      tma_prefetch_desc(&tmap_s);
-      mbar_arrive_expect_tx(q_full, C::kQBytes);
-      tma_load_3d(q_s, &tmap_q, q_full, 0, row0 * IDX_HEADS, b);
-      q_issued = true;
-      int t = 0;
+      int t = tma_issued;   // the first tiles went out during set-up
       for (; t < ntiles; ++t) {
         const int s = t % STAGES;
         if (!mbar_wait(&empty[s], ((t / STAGES) & 1) ^ 1, budget, abort_flag, p.err)) break;
@@ -206,7 +215,6 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
         const int tt = tile_of(t);
         tma_load_3d(k_s + s * kTileBytes, &tmap_k, &full[s], 0, start + tt * kTileKeys, b);
         tma_load_2d(scale_s + s * kTileKeys, &tmap_s, &full[s], start + tt * kTileKeys, b);
-        if (pf_dist && t + pf_dist < ntiles) tma_prefetch_3d(&tmap_k, 0, start + tile_of(t + pf_dist) * kTileKeys, b);
       }
       tma_issued = t;
     }
@@ -247,11 +255,12 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
     const int tok_lo = ((ew >> 2) / TSPLIT) * C::kTokPerWarp;
     const int kl = quad * 32 + lane;            // key within the tile
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-    // decode: this warp's 64 head weights in registers, packed in pairs for the
-    // f32x2 FMA; prefill (two rows per warp) reads them from shared memory
+    // W_REGS: this warp's 64 head weights (one row) in registers, packed in
+    // pairs for the f32x2 FMA; otherwise they are read from shared memory
     // (broadcast 16-byte loads) to stay within the register budget.
-    unsigned long long wp[C::kTokPerWarp == 1 ? 32 : 1];
-    if constexpr (C::kTokPerWarp == 1) {
+    static_assert(!W_REGS || C::kTokPerWarp == 1, "register weights hold one row");
+    unsigned long long wp[W_REGS ? 32 : 1];
+    if constexpr (W_REGS) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) wp[i] = pack2(w_s[tok_lo * 64 + 2 * i], w_s[tok_lo * 64 + 2 * i + 1]);
     }
@@ -271,7 +280,7 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
       for (int jj = 0; jj < C::kTokPerWarp; ++jj) {
         const int j = tok_lo + jj;
         unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
-        if constexpr (C::kTokPerWarp == 1) {
+        if constexpr (W_REGS) {
           uint32_t r0[32], r1[32];
           tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64), r0);
           tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64 + 32), r1);
@@ -405,11 +414,11 @@ int pow2_floor(int x) {
   return p;
 }
 
-template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT>
+template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT, bool W_REGS>
 int launch_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
                  const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, float* scores,
                  int64_t ld, int k, int32_t* indices, cudaStream_t stream, int score_budget_bytes) {
-  using C = Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT>;
+  using C = Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>;
   const int ntb = (n + NT - 1) / NT;
   const int64_t items = static_cast<int64_t>(B) * ntb;
   const int sms = num_sms();
@@ -440,7 +449,7 @@ int launch_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, c
   if (!make_tmap_f32_2d(&ts, k_scale_cache, static_cast<uint64_t>(T_cap), static_cast<uint64_t>(B), kTileKeys))
     return IDX_ERR_ALIGN;
 
-  auto kern = score_kernel<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT>;
+  auto kern = score_kernel<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>;
   static int configured_smem = -1;   // per instantiation
   if (configured_smem < smem) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -519,9 +528,9 @@ extern "C" int idx_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_
   if (ld <= 0) return IDX_ERR_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (n <= kDecodeRowsMax)
-    return launch_score<1, false, 6, 4, 8, 2>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
+    return launch_score<1, false, 6, 4, 8, 2, true>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
                                            scores, ld, 0, nullptr, s, 0);
-  return launch_score<4, false, 4, 2, 8, 1>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
+  return launch_score<4, false, 4, 2, 16, 1, false>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
                                          scores, ld, 0, nullptr, s, 0);
 }
 
@@ -537,9 +546,9 @@ extern "C" int idx_score_topk(const uint8_t* q_fp8, const float* w, const uint8_
   if (!indices) return IDX_ERR_NULL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (n <= kDecodeRowsMax)
-    return launch_score<1, true, 6, 4, 8, 2>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
+    return launch_score<1, true, 6, 4, 8, 2, true>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
                                           nullptr, 0, k, indices, s, 64 * 1024);
-  return launch_score<4, true, 3, 2, 8, 1>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
+  return launch_score<4, true, 3, 2, 16, 1, false>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
                                         nullptr, 0, k, indices, s, 64 * 1024);
 }
 

@@ -60,8 +60,8 @@ struct SelectSmem {
 
 // Block-wide exclusive scan of two counters.  Returns the thread's offsets; the
 // block totals land in *tot_a / *tot_b (same value in every thread).
-__device__ __forceinline__ void block_scan2(SelectSmem& sm, int a, int b, int& ea, int& eb, int& tot_a,
-                                            int& tot_b) {
+static __device__ __noinline__ void block_scan2(SelectSmem& sm, int a, int b, int& ea, int& eb, int& tot_a,
+                                         int& tot_b) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   int ia = a, ib = b;
 #pragma unroll
@@ -97,7 +97,7 @@ __device__ __forceinline__ void block_scan2(SelectSmem& sm, int a, int b, int& e
 
 // Block-wide: bins in descending order of value; find the bin that holds the
 // rem-th largest element.  Result in sm.bin, and sm.above = count in higher bins.
-__device__ __forceinline__ void find_bin(SelectSmem& sm, const uint32_t* hist, int nb, int rem) {
+static __device__ __noinline__ void find_bin(SelectSmem& sm, const uint32_t* hist, int nb, int rem) {
   const int nthr = blockDim.x;
   const int tid = threadIdx.x;
   const int per = (nb + nthr - 1) / nthr;
@@ -239,7 +239,7 @@ __device__ __forceinline__ const uint32_t* summed_hist(SelectSmem& sm, const uin
 
 // Select the kt best of a row whose keys are split over the cluster.
 //   keys[0 … nloc)  this CTA's slice (positions start … start+nloc−1), 16-byte
-//                   aligned and readable up to the next multiple of 4
+//                   aligned, and holding key 0 from nloc up to the next multiple of 4
 //   hist1           this CTA's histogram of keys >> 21 over the slice
 //   cand[0 … cap)   scratch for candidate slice indices
 //   out             the row's k output slots (global memory)
@@ -275,24 +275,24 @@ __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint3
   const bool done1 = static_cast<int>(H[b1]) == rem;
   stamp(8);
 
-  // ---- pass A: count, 4 keys per 16-byte load, branch-free predicates
+  // ---- pass A: count.  4 keys per 16-byte load, keys compared against bin
+  // edges (no shifts), no bounds test per key: the slice is padded with key 0
+  // up to a multiple of 4, and 0 lies below every bin a visible score can fall
+  // in (a finite score maps to a key ≥ 0x007FFFFF, i.e. bin ≥ 3).
   const uint4* kv = reinterpret_cast<const uint4*>(keys);
   const int nvec = (nloc + 3) >> 2;
-  const uint32_t d1 = done1 ? 1u : 0u;
+  const uint32_t lo1 = b1 << 21;              // first key of bin b1
+  const uint32_t hi1 = lo1 | 0x1FFFFFu;       // last key of bin b1
+  // done1: everything from bin b1 up is selected; otherwise keys above bin b1
+  // are selected and keys inside it become candidates
+  const uint32_t sel_above = done1 ? lo1 - 1u : hi1;
   int cg = 0, ce = 0;
   for (int v = tid; v < nvec; v += nthr) {
     const uint4 q = kv[v];
-    const uint32_t kk[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t valid = (4 * v + e < nloc) ? 1u : 0u;
-      const uint32_t top = kk[e] >> 21;
-      const uint32_t eq = (top == b1) ? 1u : 0u;
-      cg += static_cast<int>(valid & (((top > b1) ? 1u : 0u) | (d1 & eq)));
-      ce += static_cast<int>(valid & (d1 ^ 1u) & eq);
-    }
+    cg += (q.x > sel_above) + (q.y > sel_above) + (q.z > sel_above) + (q.w > sel_above);
+    ce += (q.x >= lo1) + (q.y >= lo1) + (q.z >= lo1) + (q.w >= lo1);
   }
-  stamp(9);
+  ce = done1 ? 0 : ce - cg;                   // keys inside bin b1
   int og, oe, tg, te;
   block_scan2(sm, cg, ce, og, oe, tg, te);
   if (tid == 0) sm.cta_cnt[0][0] = tg;
@@ -303,22 +303,19 @@ __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint3
   // ---- pass A: write
   {
     int wg = sm.cta_base[0] + og, we = oe;
-    const uint32_t keep = overflow ? 0u : 1u;
+    const bool keep = !overflow && !done1;
     for (int v = tid; v < nvec; v += nthr) {
       const uint4 q = kv[v];
       const uint32_t kk[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int i = 4 * v + e;
-        const uint32_t valid = (i < nloc) ? 1u : 0u;
-        const uint32_t top = kk[e] >> 21;
-        const uint32_t eq = (top == b1) ? 1u : 0u;
-        const uint32_t g = valid & (((top > b1) ? 1u : 0u) | (d1 & eq));
-        const uint32_t c = valid & (d1 ^ 1u) & eq & keep;
+        const bool g = kk[e] > sel_above;
+        const bool c = keep && !g && kk[e] >= lo1;
         if (g) ro.put(wg, start + i);
         if (c) cand[we] = i;
-        wg += static_cast<int>(g);
-        we += static_cast<int>(c);
+        wg += g ? 1 : 0;
+        we += c ? 1 : 0;
       }
     }
   }

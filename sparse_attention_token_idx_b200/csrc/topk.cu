@@ -73,6 +73,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
       }
     }
   }
+  // pad the slice with key 0 up to a multiple of 4 (the selection reads whole vectors)
+  if (threadIdx.x < 4 && nloc + static_cast<int>(threadIdx.x) < ((nloc + 3) & ~3)) sc_s[nloc + threadIdx.x] = 0u;
   __syncthreads();
   if (tr && threadIdx.x == 0) tr[3] = globaltimer_ns();
   int32_t* out = p.indices + row * p.k;
