@@ -147,21 +147,26 @@ IDX_API int idx_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cac
  *   indices [B, n, k] int32 out: the k_t = min(k, visible(b,i)) positions with the
  *   highest scores, in unspecified order, in columns 0 … k_t−1; columns k_t … k−1
  *   hold −1.  Ties at the k_t-th score are broken arbitrarily.
- *   max_len as in idx_score (and ≤ ld).  ws / ws_bytes: reserved, pass NULL / 0.
+ *   max_len as in idx_score (and ≤ ld).  ws / ws_bytes: not used, pass NULL / 0.
  */
 IDX_API int idx_topk(const float* scores, const int32_t* lengths, int B, int n, int64_t ld, int max_len, int causal, int k,
              int32_t* indices, void* ws, size_t ws_bytes, idx_stream_t stream);
 
 /*
- * idx_score_topk — idx_score followed by idx_topk in one kernel: the scores of
- * a row never leave on-chip memory.  Arguments as in idx_score / idx_topk.
+ * idx_score_topk — scores and top-k in one call, arguments as in idx_score /
+ * idx_topk.  Decode-shaped calls (n ≤ 2) run one kernel in which a row's scores
+ * never leave on-chip memory.  Prefill-shaped calls (n > 2) given a workspace of
+ * at least idx_workspace_size(B, n, max_len, k) bytes (16-byte aligned) write
+ * the scores there and select with the top-k kernel (faster: selections of
+ * different rows overlap); without one they use the single-kernel path.
  */
 IDX_API int idx_score_topk(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
                    const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, int k,
                    int32_t* indices, void* ws, size_t ws_bytes, idx_stream_t stream);
 
-/* Scratch bytes idx_topk / idx_score_topk need for these sizes (currently 0). */
-IDX_API size_t idx_workspace_size(int B, int n, int T_cap, int k);
+/* Workspace bytes idx_score_topk uses for these sizes: 0 for decode-shaped
+ * calls (n ≤ 2), B·n·max_len·4 (fp32 scores) for prefill-shaped ones. */
+IDX_API size_t idx_workspace_size(int B, int n, int max_len, int k);
 
 /*
  * idx_status — synchronises `stream`, then reads and clears the device error

@@ -166,17 +166,25 @@ def topk(scores, lengths, causal: bool, k: int, max_len: int, out=None, stream=N
     return out
 
 
+def workspace_size(B: int, n: int, max_len: int, k: int) -> int:
+    return int(load().idx_workspace_size(B, n, max_len, k))
+
+
 def score_topk(q_fp8, w, k_cache, k_scale_cache, lengths, causal: bool, k: int, max_len: int, out=None,
-               stream=None):
-    """Fused scores + top-k: positions [B, n, k] int32 (a set per row, −1 padded)."""
+               ws: torch.Tensor | None = None, stream=None):
+    """Scores + top-k: positions [B, n, k] int32 (a set per row, −1 padded).
+    ``ws`` (a uint8 CUDA tensor of workspace_size() bytes) is used by
+    prefill-shaped calls; decode-shaped calls need none."""
     B, n = q_fp8.shape[0], q_fp8.shape[1]
     T_cap = k_cache.shape[1]
     out = out if out is not None else torch.empty((B, n, k), dtype=torch.int32, device=q_fp8.device)
+    ws_ptr, ws_bytes = (None, 0) if ws is None else (_ptr(ws, None, "ws"), ws.numel() * ws.element_size())
     _check(load().idx_score_topk(_ptr(q_fp8, torch.uint8, "q_fp8"), _ptr(w, torch.float32, "w"),
                                  _ptr(k_cache, torch.uint8, "k_cache"),
                                  _ptr(k_scale_cache, torch.float32, "k_scale"),
                                  _ptr(lengths, torch.int32, "lengths"), B, n, T_cap, max_len, int(causal), k,
-                                 _ptr(out, torch.int32, "indices"), None, 0, _stream(stream)), "idx_score_topk")
+                                 _ptr(out, torch.int32, "indices"), ws_ptr, ws_bytes, _stream(stream)),
+           "idx_score_topk")
     return out
 
 

@@ -185,12 +185,12 @@ extern "C" const char* idx_error_string(int code) {
   }
 }
 
-extern "C" size_t idx_workspace_size(int B, int n, int T_cap, int k) {
-  (void)B;
-  (void)n;
-  (void)T_cap;
+extern "C" size_t idx_workspace_size(int B, int n, int max_len, int k) {
   (void)k;
-  return 0;
+  if (B <= 0 || n <= 0 || max_len <= 0) return 0;
+  if (n <= 2) return 0;   // decode-shaped calls select in shared memory
+  // prefill-shaped calls: one fp32 score row of max_len columns per query row
+  return static_cast<size_t>(B) * static_cast<size_t>(n) * static_cast<size_t>(max_len) * sizeof(float);
 }
 
 extern "C" void idx_debug_set(unsigned int flags, unsigned long long budget_ns) {

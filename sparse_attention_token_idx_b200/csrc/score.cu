@@ -349,7 +349,15 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
       for (int j = 0; j < NT; ++j) {
         if (!row_exists(j)) continue;
         float* row = p.scores + (static_cast<int64_t>(b) * p.n + row0 + j) * p.ld;
-        for (int64_t c = lo + threadIdx.x; c < share_hi; c += blockDim.x) row[c] = -INFINITY;
+        // scalar head up to a 16-byte boundary, 16-byte stores, scalar tail
+        const int64_t head = (4 - ((reinterpret_cast<uintptr_t>(row + lo) >> 2) & 3)) & 3;
+        const int64_t body_lo = lo + (head < share_hi - lo ? head : share_hi - lo);
+        const int64_t nvec = (share_hi - body_lo) >> 2;
+        for (int64_t c = lo + threadIdx.x; c < body_lo; c += blockDim.x) row[c] = -INFINITY;
+        float4* rv = reinterpret_cast<float4*>(row + body_lo);
+        const float4 ninf = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) rv[v] = ninf;
+        for (int64_t c = body_lo + 4 * nvec + threadIdx.x; c < share_hi; c += blockDim.x) row[c] = -INFINITY;
       }
     }
   } else {
@@ -538,13 +546,24 @@ extern "C" int idx_score_topk(const uint8_t* q_fp8, const float* w, const uint8_
                               const float* k_scale_cache, const int32_t* lengths, int B, int n, int T_cap,
                               int max_len, int causal, int k, int32_t* indices, void* ws, size_t ws_bytes,
                               idx_stream_t stream) {
-  (void)ws;
-  (void)ws_bytes;
   const int c = check_score_args(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal);
   if (c <= 0) return c;
   if (k <= 0) return IDX_ERR_K;
   if (!indices) return IDX_ERR_NULL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // Prefill-shaped calls with a workspace: scores of all rows to the workspace
+  // (the tcgen05 scorer at full tensor throughput), then the top-k kernel with
+  // several rows per SM in flight.  A row's selection then overlaps other rows'
+  // work instead of stalling its CTA's MMA pipeline.
+  const size_t need = idx_workspace_size(B, n, max_len, k);
+  if (n > kDecodeRowsMax && ws && ws_bytes >= need && need > 0) {
+    if (reinterpret_cast<uintptr_t>(ws) & 15) return IDX_ERR_ALIGN;
+    float* scores = static_cast<float*>(ws);
+    const int r = launch_score<4, false, 4, 2, 16, 1, false>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap,
+                                                             max_len, causal, scores, max_len, 0, nullptr, s, 0);
+    if (r != IDX_OK) return r;
+    return idx_topk(scores, lengths, B, n, max_len, max_len, causal, k, indices, nullptr, 0, stream);
+  }
   if (n <= kDecodeRowsMax)
     return launch_score<1, true, 6, 4, 8, 2, true>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
                                           nullptr, 0, k, indices, s, 64 * 1024);

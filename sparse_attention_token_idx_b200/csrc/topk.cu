@@ -16,16 +16,25 @@ namespace idx {
 namespace {
 
 constexpr int kTopkThreads = 256;
-constexpr int kTopkCand = 4096;   // candidate list entries
+constexpr int kTopkCandMax = 4096;   // candidate list entries (at most)
 
 constexpr int kTraceSlotsT = 16;
+
+// Candidates are the keys of the threshold bin of the level-1 histogram, a
+// small part of a row; a quarter of the slice (1024 … 4096 entries) holds
+// them, and a list that overflows falls back to scanning the slice.
+int topk_cand_cap(int chunk_cap) {
+  int c = chunk_cap / 4;
+  c = c < 1024 ? 1024 : c;
+  return c > kTopkCandMax ? kTopkCandMax : c;
+}
 
 struct TopkParams {
   const float* scores;
   const int32_t* lengths;
   int32_t* indices;
   int64_t ld;
-  int B, n, max_len, causal, k, G, chunk_cap;
+  int B, n, max_len, causal, k, G, chunk_cap, cand_cap;
   unsigned int* err;
   unsigned long long* trace;   // per-CTA phase stamps, or null
 };
@@ -36,7 +45,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   SelectSmem& sel = *reinterpret_cast<SelectSmem*>(smem);
   uint32_t* hist1 = reinterpret_cast<uint32_t*>(smem + sizeof(SelectSmem));
   int* cand = reinterpret_cast<int*>(smem + sizeof(SelectSmem) + kHistBins * 4);
-  uint32_t* sc_s = reinterpret_cast<uint32_t*>(smem + sizeof(SelectSmem) + kHistBins * 4 + kTopkCand * 4);
+  uint32_t* sc_s = reinterpret_cast<uint32_t*>(smem + sizeof(SelectSmem) + kHistBins * 4 + p.cand_cap * 4);
   unsigned long long* tr = (p.trace && blockIdx.x < 8192) ? p.trace + blockIdx.x * kTraceSlotsT : nullptr;
   if (tr && threadIdx.x == 0) tr[0] = globaltimer_ns();
   const uint32_t rank = cluster_rank();
@@ -52,6 +61,16 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   const int start = static_cast<int>(rank) * chunk;
   const int nloc = max(0, min(start + chunk, vis) - start);
   const float* src = p.scores + row * p.ld + start;
+  int32_t* out = p.indices + row * p.k;
+  const int kt = min(p.k, vis);
+  if (kt == vis) {
+    // every visible position is selected: no scores needed, slot s holds position s
+    for (int t = threadIdx.x; t < nloc; t += blockDim.x) out[start + t] = start + t;
+    if (rank == 0)
+      for (int t = kt + threadIdx.x; t < p.k; t += blockDim.x) out[t] = -1;
+    if (tr && threadIdx.x == 0) tr[4] = globaltimer_ns();
+    return;   // uniform over the cluster (same vis): no CTA waits at a cluster barrier
+  }
   for (int t = threadIdx.x; t < kHistBins; t += blockDim.x) hist1[t] = 0;
   __syncthreads();
   // four independent loads in flight per thread
@@ -77,13 +96,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   if (threadIdx.x < 4 && nloc + static_cast<int>(threadIdx.x) < ((nloc + 3) & ~3)) sc_s[nloc + threadIdx.x] = 0u;
   __syncthreads();
   if (tr && threadIdx.x == 0) tr[3] = globaltimer_ns();
-  int32_t* out = p.indices + row * p.k;
-  const int kt = min(p.k, vis);
-  if (kt == vis) {
-    for (int t = threadIdx.x; t < nloc; t += blockDim.x) out[start + t] = start + t;
-  } else {
-    cluster_select_row(sel, sc_s, nloc, start, kt, hist1, cand, kTopkCand, out, G, rank, tr);
-  }
+  cluster_select_row(sel, sc_s, nloc, start, kt, hist1, cand, p.cand_cap, out, G, rank, tr);
   if (rank == 0)
     for (int t = kt + threadIdx.x; t < p.k; t += blockDim.x) out[t] = -1;
   if (G > 1) cluster_sync();
@@ -119,7 +132,8 @@ extern "C" int idx_topk(const float* scores, const int32_t* lengths, int B, int 
   const int budget = 64 * 1024;
   while (G < 8 && static_cast<int64_t>((max_len + G - 1) / G) * 4 > budget) G *= 2;
   const int chunk_cap = ((max_len + G - 1) / G + 3) / 4 * 4;   // whole 16-byte vectors
-  const int smem = 128 + static_cast<int>(sizeof(SelectSmem)) + (kHistBins + kTopkCand) * 4 + chunk_cap * 4;
+  const int cand_cap = topk_cand_cap(chunk_cap);
+  const int smem = 128 + static_cast<int>(sizeof(SelectSmem)) + (kHistBins + cand_cap) * 4 + chunk_cap * 4;
   if (smem > max_dynamic_smem()) return IDX_ERR_SHAPE;
   if (rows * G > 0x7FFFFFFF) return IDX_ERR_SHAPE;
   static int configured = -1;
@@ -128,7 +142,7 @@ extern "C" int idx_topk(const float* scores, const int32_t* lengths, int B, int 
       return check_launch();
     configured = smem;
   }
-  TopkParams p{scores, lengths, indices, ld, B, n, max_len, causal, k, G, chunk_cap, device_error_word(),
+  TopkParams p{scores, lengths, indices, ld, B, n, max_len, causal, k, G, chunk_cap, cand_cap, device_error_word(),
                (debug_state().flags & 2u) ? trace_buffer() : nullptr};
   if (!p.err) return check_launch();
   cudaLaunchConfig_t cfg = {};

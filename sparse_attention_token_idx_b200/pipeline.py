@@ -43,8 +43,10 @@ class Indexer:
         X.quant_queries_append(q, w_raw, k_new, positions, self.k_cache, self.k_scale_cache, self.fmt, q_fp8, w,
                                stream=stream)
         out = out if out is not None else self._buf("idx", (B, n, self.k), torch.int32)
+        ws_bytes = X.workspace_size(B, n, max_len, self.k)
+        ws = self._buf("ws", (ws_bytes,), torch.uint8) if ws_bytes else None
         return X.score_topk(q_fp8, w, self.k_cache, self.k_scale_cache, lengths, causal, self.k, max_len,
-                            out=out, stream=stream)
+                            out=out, ws=ws, stream=stream)
 
     def capture(self, k_new, q, w_raw, positions, lengths, *, causal: bool, max_len: int):
         """Record one step on static input tensors into a CUDA graph; returns

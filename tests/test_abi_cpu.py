@@ -36,7 +36,8 @@ def test_error_strings_without_gpu():
     lib = binding.load()
     assert lib.idx_error_string(0) == b"ok"
     assert b"NULL" in lib.idx_error_string(-1)
-    assert lib.idx_workspace_size(128, 1, 16384, 2048) == 0
+    assert lib.idx_workspace_size(128, 1, 16384, 2048) == 0          # decode: selection in shared memory
+    assert lib.idx_workspace_size(2, 2048, 16384, 2048) == 2 * 2048 * 16384 * 4   # prefill: fp32 score rows
 
 
 def test_host_argument_checks_run_before_any_device_work():

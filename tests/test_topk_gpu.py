@@ -54,14 +54,21 @@ FUSED = [
 ]
 
 
+@pytest.mark.parametrize("use_ws", [False, True])
 @pytest.mark.parametrize("name,B,n,positions,T_cap,causal,fmt,k", FUSED)
-def test_fused_topk_matches_oracle_and_unfused(name, B, n, positions, T_cap, causal, fmt, k):
+def test_fused_topk_matches_oracle_and_unfused(name, B, n, positions, T_cap, causal, fmt, k, use_ws):
     from sparse_attention_token_idx_b200 import binding as X
     case = synth.make_case(name, 300 + len(name), B, n, positions, T_cap=T_cap, causal=causal, fmt=fmt, k=k)
     kc, ks, lengths = gpu_state(case)
     qc, w = gpu_queries(case)
     max_len = int(case.lengths.max())
-    idx = X.score_topk(qc, w, kc, ks, lengths, causal, k, max_len).cpu().numpy()
+    ws = None
+    if use_ws:
+        nbytes = X.workspace_size(B, n, max_len, k)
+        if nbytes == 0:
+            pytest.skip("decode-shaped calls use no workspace")
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    idx = X.score_topk(qc, w, kc, ks, lengths, causal, k, max_len, ws=ws).cpu().numpy()
     sc = X.score(qc, w, kc, ks, lengths, causal, max_len, ld=max_len).cpu().numpy()
     assert X.status() == (0, 0)
     okc, oks = oracle_state(case)
