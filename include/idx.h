@@ -68,7 +68,8 @@ enum idx_status_code {
   IDX_ERR_LAUNCH = -6,      /* the CUDA launch failed (the CUDA error is in idx_last_cuda_error) */
   IDX_ERR_DEVICE = -7,      /* idx_status: a kernel set the device error word */
   IDX_ERR_CUDA = -8,        /* idx_status: the stream itself reported a CUDA error */
-  IDX_ERR_UNSUPPORTED = -9  /* no device code for this GPU (not sm_100) */
+  IDX_ERR_UNSUPPORTED = -9, /* no device code for this GPU (not sm_100) */
+  IDX_ERR_SCRATCH = -10     /* idx_score_topk_noalloc: the call needs more than the library's fixed scratch */
 };
 
 /* Bits of the device error word (returned by idx_device_error_bits). */
@@ -163,6 +164,26 @@ IDX_API int idx_topk(const float* scores, const int32_t* lengths, int B, int n, 
 IDX_API int idx_score_topk(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
                    const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, int k,
                    int32_t* indices, void* ws, size_t ws_bytes, idx_stream_t stream);
+
+/*
+ * idx_score_topk_noalloc — idx_score_topk for callers that cannot allocate
+ * device memory when they call (for example while their stream is being
+ * captured into a CUDA graph, or inside a plugin enqueue step that must not
+ * allocate).  The pages have no counterpart: this is a deployment variant.
+ * Prefill-shaped calls keep their score workspace in a buffer the library
+ * owns: a file-scope device array of 64 MiB (B·n·max_len ≤ 16 Mi scores),
+ * held on every GPU that loads the library until the process exits.  Larger
+ * calls return IDX_ERR_SCRATCH; decode-shaped calls need no scratch.
+ *   - The first call on a device looks up the buffer's device address (no
+ *     allocation); make that first call before any stream capture.
+ *   - Every call reuses the same buffer and rewrites all of the part it uses,
+ *     so nothing needs clearing, but calls that overlap on the GPU (other
+ *     streams, other threads) race on it: serialise them.
+ *   - It calls no cudaMalloc / cudaFree; arguments otherwise as idx_score_topk.
+ */
+IDX_API int idx_score_topk_noalloc(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache,
+                                   const float* k_scale_cache, const int32_t* lengths, int B, int n, int T_cap,
+                                   int max_len, int causal, int k, int32_t* indices, idx_stream_t stream);
 
 /* Workspace bytes idx_score_topk uses for these sizes: 0 for decode-shaped
  * calls (n ≤ 2), B·n·max_len·4 (fp32 scores) for prefill-shaped ones. */

@@ -38,6 +38,7 @@ SIGNATURES = {
     "idx_score": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P]),
     "idx_topk": (_I, [_P, _P, _I, _I, _I64, _I, _I, _I, _P, _P, _SZ, _P]),
     "idx_score_topk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
+    "idx_score_topk_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
     "idx_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "idx_status": (_I, [_P]),
     "idx_device_error_bits": (ctypes.c_uint, []),

@@ -20,6 +20,7 @@
 // left at a cluster barrier.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 #include "api_internal.h"
@@ -586,3 +587,59 @@ unsigned long long* trace_buffer() {
   return static_cast<unsigned long long*>(ptr);
 }
 }  // namespace idx
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the prefill-shaped score + top-k.
+//
+// Some callers cannot allocate device memory at the moment they call in — for
+// example code that enqueues work while its stream is being captured into a
+// CUDA graph, or an inference-engine plugin whose enqueue step is not allowed
+// to allocate.  They cannot provide the score workspace idx_score_topk uses
+// for prefill-shaped calls, so this entry point keeps that workspace in a
+// fixed buffer owned by the library.
+namespace idx {
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;   // 64 MiB: B·n·max_len ≤ 16 Mi scores
+static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / sizeof(float)];
+
+std::atomic<float*> g_static_scratch_addr[64];
+
+// Device address of g_static_scratch on the current device (host code cannot
+// use the symbol itself: on the host it only names a stand-in).
+float* static_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  float* a = g_static_scratch_addr[dev].load();
+  if (!a) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return nullptr;
+    a = static_cast<float*>(ptr);
+    g_static_scratch_addr[dev].store(a);
+  }
+  return a;
+}
+
+}  // namespace
+}  // namespace idx
+
+extern "C" int idx_score_topk_noalloc(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache,
+                                      const float* k_scale_cache, const int32_t* lengths, int B, int n, int T_cap,
+                                      int max_len, int causal, int k, int32_t* indices, idx_stream_t stream) {
+  const int c = check_score_args(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal);
+  if (c <= 0) return c;
+  if (k <= 0) return IDX_ERR_K;
+  if (!indices) return IDX_ERR_NULL;
+  const size_t need = idx_workspace_size(B, n, max_len, k);
+  if (need > kStaticScratchBytes) return IDX_ERR_SCRATCH;
+  if (need == 0)   // decode-shaped: the single kernel needs no scratch
+    return idx_score_topk(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal, k, indices,
+                          nullptr, 0, stream);
+  float* scratch = static_scratch();
+  if (!scratch) {
+    check_launch();   // records the CUDA error of the failed lookup
+    return IDX_ERR_LAUNCH;
+  }
+  return idx_score_topk(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal, k, indices,
+                        scratch, kStaticScratchBytes, stream);
+}
