@@ -70,7 +70,9 @@ struct Cfg {
   static constexpr int kTokPerWarp = NT / kTokGroups;
   static constexpr int kWarpsPerTile = EPI_WARPS / TSPLIT;   // warps that consume one tile
   static constexpr int kQBytes = N * IDX_DIM;
-  static constexpr int kCand = NT == 1 ? 4096 : 1024;     // candidate list of the select
+  static constexpr int kCand = NT == 1 ? 4096 : 1024;     // scratch ints of the select
+  // one row per CTA: 16-bit entries of the scratch that hold the production-time list
+  static constexpr int kList = (FUSED && NT == 1) ? 6144 : 0;
   // shared memory carve (offsets from a 1024-aligned base)
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
@@ -116,6 +118,7 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
   SelectSmem& sel = *reinterpret_cast<SelectSmem*>(smem + C::kOffSel);
   uint32_t* hist1 = reinterpret_cast<uint32_t*>(smem + C::kOffHist1);
   int* cand = reinterpret_cast<int*>(smem + C::kOffCand);
+  uint16_t* list16 = reinterpret_cast<uint16_t*>(cand);   // first C::kList entries of the scratch
   uint32_t* sc_s = reinterpret_cast<uint32_t*>(smem + C::kOffScores);
 
   const int warp = threadIdx.x >> 5;
@@ -168,6 +171,7 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
     mbar_init(drain_bar, 1);
     mbar_init(never_bar, 1);
     *abort_flag = 0;
+    if constexpr (FUSED) row_filter_reset(sel);
     fence_barrier_init();
     // Thread 0 is also the TMA producer: start the query and the first STAGES
     // key tiles now, so that their DRAM latency overlaps the rest of the set-up
@@ -195,8 +199,10 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
     const int tok = row0 + j;
     w_s[i] = (tok < p.n && !bad) ? p.w[(static_cast<int64_t>(b) * p.n + tok) * IDX_HEADS + (i % IDX_HEADS)] : 0.f;
   }
-  if constexpr (FUSED)
+  if constexpr (FUSED) {
     for (int i = threadIdx.x; i < NT * kHistBins; i += blockDim.x) hist1[i] = 0;
+    if constexpr (NT == 1) select_prepare(sel);   // one row: the selection state is set up here
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -323,7 +329,13 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
         if constexpr (FUSED) {
           const uint32_t u = order_key(sc);
           sc_s[j * p.chunk_cap + tt * kTileKeys + kl] = visible ? u : 0u;
-          if (visible) atomicAdd(&hist1[j * kHistBins + (u >> 21)], 1u);
+          if (visible) {
+            if constexpr (NT == 1) select_count_key(sel, hist1, u);   // with the coarse sums
+            else atomicAdd(&hist1[j * kHistBins + (u >> 21)], 1u);
+          }
+          // one row per CTA: keys that may reach the top k go to the short list
+          if constexpr (C::kList > 0)
+            if (G == 1) row_filter_append(sel, list16, C::kList, u, visible, tt * kTileKeys + kl);
         } else {
           if (row_exists(j) && key < p.ld) {
             p.scores[(static_cast<int64_t>(b) * p.n + row0 + j) * p.ld + key] = visible ? sc : -INFINITY;
@@ -335,6 +347,14 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
       if (lane == 0) {
         mbar_arrive(&acc_empty[a]);
         mbar_arrive(&empty[s]);
+      }
+      // the first epilogue warp raises the list's bound after tile 4 and every 8 tiles
+      if constexpr (C::kList > 0) {
+        if (G == 1 && ew == 0 && (t == 4 || (t >= 8 && (t & 7) == 0))) {
+          const int v0 = row_vis(0);
+          const int target = row_filter_target((t + 1) * kTileKeys, v0, min(p.k, v0));
+          if (target > 0) row_filter_raise(sel, hist1, target);
+        }
       }
     }
   }
@@ -381,7 +401,8 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
       } else {
         if (trace && j == 0 && threadIdx.x == 0) tr[6] = globaltimer_ns();
         cluster_select_row(sel, sc_s + j * p.chunk_cap, nloc, start, kt, hist1 + j * kHistBins, cand, C::kCand,
-                           out, G, rank, (trace && j == 0) ? tr : nullptr, const_cast<const int*>(abort_flag));
+                           C::kList, NT == 1, out, G, rank, (trace && j == 0) ? tr : nullptr,
+                           const_cast<const int*>(abort_flag));
         if (rank == 0)
           for (int i = kt + threadIdx.x; i < p.k; i += blockDim.x) out[i] = -1;
       }

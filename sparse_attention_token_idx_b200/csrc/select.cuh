@@ -43,7 +43,7 @@ struct Grp {
   }
 };
 
-struct SelectSmem {
+struct alignas(16) SelectSmem {
   uint32_t hist[kHistBins];      // this CTA's level-2 histogram
   uint32_t hist3[kHistBins / 2]; // this CTA's level-3 histogram (own buffer: one barrier per exchange)
   uint32_t hsum[kHistBins];      // cluster-summed histogram
@@ -55,6 +55,11 @@ struct SelectSmem {
   int cta_base[2];               // cluster prefix of those totals for this CTA
   int any_abort;
   int pad[3];
+  uint32_t coarse[3][64];        // one-CTA path: coarse histograms (32 fine bins per entry) of levels 1-3
+  uint32_t ctr_gc;               // one-CTA path: output slots taken (low 16 bits) | bin-b1 keys listed (high)
+  uint32_t ctr_tie;              // one-CTA path: ties at the 32-bit threshold seen
+  uint32_t filt_lo;              // row filter: keys below this bound are not listed
+  int list_cnt;                  // row filter: list entries taken
   int32_t out_s[kStage];         // staged positions of the current row (CTA 0's copy is the one used)
 };
 
@@ -433,15 +438,418 @@ __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint3
   flush_row<CL>(sm, ro, kt, rank);
 }
 
+// ---------------------------------------------------------------------------
+// One-CTA selection.
+//
+// A row held by a single CTA is selected with the same 11 + 11 + 10-bit
+// refinement, arranged for few barriers and little work per key:
+//   - while the scores are produced, the level-1 histogram and its coarse sums
+//     (32 bins per entry) are counted, and keys at or above a running lower
+//     bound of the level-1 threshold bin go to a short index list
+//     (row_filter_append / row_filter_raise).  After the last score the exact
+//     bin b1 says whether the list is complete (b1 at or above the last bound);
+//     pass A then visits the list, otherwise the whole slice;
+//   - every warp finds a threshold bin on its own (no barrier): a prefix over
+//     the coarse histogram picks an entry, a prefix over its 32 fine bins
+//     picks the bin; all warps read the same histograms;
+//   - a pass gives each warp a contiguous segment of the items; a lane counts
+//     its items, the warp scans the lane counts and reserves its output range
+//     with one shared atomic, and each lane writes its items as one run — no
+//     barrier inside a pass.  The level-2 and level-3 histograms are counted
+//     in the pass before the level that reads them.
+// Barriers per row after the scores: 1 (threshold in the top 11 bits), 2 (22
+// bits), 3 (32 bits), plus one before the first level when the caller did not
+// prepare the state (select_prepare).  Output order is unspecified (a set).
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Zero the level-2/3 histograms, their coarse sums, the level-1 coarse sums
+// and the pass counters (block-wide; a barrier must follow before use).
+__device__ __forceinline__ void select_prepare(SelectSmem& sm) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  for (int i = tid; i < kHistBins / 4; i += nthr) reinterpret_cast<uint4*>(sm.hist)[i] = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = tid; i < kHistBins / 8; i += nthr) reinterpret_cast<uint4*>(sm.hist3)[i] = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = tid; i < 3 * 64; i += nthr) sm.coarse[i / 64][i % 64] = 0u;
+  if (tid == 0) {
+    sm.ctr_gc = 0u;
+    sm.ctr_tie = 0u;
+  }
+}
+
+// Bins in descending order of key; the bin holding the rem-th largest key
+// (rem ≥ 1) and the number of keys in higher bins.  NB fine bins, NB/32
+// coarse entries (64 or 32).  Warp-collective.
+template <int NB>
+__device__ __forceinline__ void warp_find_bin(const uint32_t* hist, const uint32_t* coarse, int rem, int& bin,
+                                              int& above) {
+  constexpr int NC = NB / 32;
+  static_assert(NC == 64 || NC == 32, "coarse histogram of 32 or 64 entries");
+  const int lane = threadIdx.x & 31;
+  int c0, c1 = 0;   // lane's coarse entries, higher one first
+  if constexpr (NC == 64) {
+    const uint2 v = *reinterpret_cast<const uint2*>(coarse + NC - 2 - 2 * lane);
+    c0 = static_cast<int>(v.y);
+    c1 = static_cast<int>(v.x);
+  } else {
+    c0 = static_cast<int>(coarse[NC - 1 - lane]);
+  }
+  const int s = c0 + c1;
+  int inc = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  const uint32_t hit = __ballot_sync(0xFFFFFFFFu, inc >= rem);
+  if (hit == 0u) {   // fewer than rem keys in the histogram: not reachable with valid counts
+    bin = 0;
+    above = 0;
+    return;
+  }
+  const int L = __ffs(hit) - 1;
+  const int exc = inc - s;
+  const bool first = exc + c0 >= rem;
+  int sup = NC == 64 ? (first ? NC - 1 - 2 * lane : NC - 2 - 2 * lane) : NC - 1 - lane;
+  int sup_above = first ? exc : exc + c0;
+  sup = __shfl_sync(0xFFFFFFFFu, sup, L);
+  sup_above = __shfl_sync(0xFFFFFFFFu, sup_above, L);
+  const int h = static_cast<int>(hist[sup * 32 + 31 - lane]);
+  int inc2 = h;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xFFFFFFFFu, inc2, o);
+    if (lane >= o) inc2 += t;
+  }
+  const uint32_t hit2 = __ballot_sync(0xFFFFFFFFu, sup_above + inc2 >= rem);
+  const int J = hit2 ? __ffs(hit2) - 1 : 31;   // the coarse entry guarantees a hit
+  bin = sup * 32 + 31 - J;
+  above = sup_above + __shfl_sync(0xFFFFFFFFu, inc2 - h, J);
+}
+
+// Production side, per key: level-1 histogram and its coarse sums.
+__device__ __forceinline__ void select_count_key(SelectSmem& sm, uint32_t* hist1, uint32_t key) {
+  atomicAdd(&hist1[key >> 21], 1u);
+  atomicAdd(&sm.coarse[0][key >> 26], 1u);
+}
+
+// Production side of the row filter, warp-collective (all 32 lanes, each with
+// its own key): visible keys at or above the current bound are appended to the
+// list at slice index idx.  Entries past the capacity are dropped (the count
+// still grows, which marks the list incomplete).
+__device__ __forceinline__ void row_filter_append(SelectSmem& sm, uint16_t* list, int cap, uint32_t key,
+                                                  bool visible, int idx) {
+  const uint32_t lo = *reinterpret_cast<const volatile uint32_t*>(&sm.filt_lo);
+  const bool p = visible && key >= lo;
+  const uint32_t m = __ballot_sync(0xFFFFFFFFu, p);
+  if (m == 0u) return;
+  int base = 0;
+  if ((threadIdx.x & 31) == 0) base = atomicAdd(&sm.list_cnt, __popc(m));
+  base = __shfl_sync(0xFFFFFFFFu, base, 0);
+  const int pos = base + __popc(m & lanemask_lt());
+  if (p && pos < cap) list[pos] = static_cast<uint16_t>(idx);
+}
+
+// Raise the bound, one warp (warp-collective): the highest bin L such that at
+// least `target` of the keys counted so far lie in bins ≥ L.  Other warps may
+// still be adding to the histograms; every count read is at most its final
+// value, so L never exceeds what the keys seen so far support.
+__device__ __forceinline__ void row_filter_raise(SelectSmem& sm, const uint32_t* hist1, int target) {
+  int bin, above;
+  warp_find_bin<kHistBins>(hist1, sm.coarse[0], target, bin, above);
+  // a miss (fewer than target keys counted) or a racy read leaves bin 0: no raise
+  if ((threadIdx.x & 31) == 0) {
+    const uint32_t lo = static_cast<uint32_t>(bin) << 21;
+    if (lo > sm.filt_lo) sm.filt_lo = lo;
+  }
+}
+
+// Target count for row_filter_raise after m of a row's vis keys: 1.5 × the
+// expected share of the kt best among them, plus a margin; 0 = do not raise.
+__device__ __forceinline__ int row_filter_target(int m, int vis, int kt) {
+  if (vis <= 0 || m <= 0) return 0;
+  const int t = static_cast<int>(1.5f * static_cast<float>(kt) * static_cast<float>(m) / static_cast<float>(vis)) + 32;
+  return t < m ? t : 0;
+}
+
+// Reset the row filter (one thread; a barrier must follow before production).
+__device__ __forceinline__ void row_filter_reset(SelectSmem& sm) {
+  sm.filt_lo = 0u;
+  sm.list_cnt = 0;
+}
+
+// Items of a pass: entries of a 16-bit index list, or the slice itself (key 0
+// past nloc).  A lane takes 4 consecutive items per step.
+struct PassItems {
+  const uint32_t* keys;
+  const uint16_t* list;   // null: the slice
+  int n;                  // list entries, or slice length rounded up to 4
+  __device__ __forceinline__ void fetch(int i0, uint32_t (&kk)[4], int (&ix)[4]) const {
+    if (list) {
+      const uint2 e = *reinterpret_cast<const uint2*>(list + i0);
+      ix[0] = static_cast<int>(e.x & 0xFFFFu);
+      ix[1] = static_cast<int>(e.x >> 16);
+      ix[2] = static_cast<int>(e.y & 0xFFFFu);
+      ix[3] = static_cast<int>(e.y >> 16);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) kk[u] = i0 + u < n ? keys[ix[u]] : 0u;
+    } else {
+      const uint4 q = *reinterpret_cast<const uint4*>(keys + i0);
+      kk[0] = q.x;
+      kk[1] = q.y;
+      kk[2] = q.z;
+      kk[3] = q.w;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) ix[u] = i0 + u;
+    }
+  }
+};
+
+// This warp's segment of a pass over n items (4-aligned bounds).
+__device__ __forceinline__ void warp_segment(int n, int& beg, int& end) {
+  const int nw = static_cast<int>(blockDim.x >> 5), warp = static_cast<int>(threadIdx.x >> 5);
+  const int seg = ((n + nw - 1) / nw + 3) & ~3;
+  beg = warp * seg;
+  end = min(n, beg + seg);
+}
+
+// Warp-collective: reserve this warp's range of a pass from a shared counter
+// (packed counts allowed: fields never carry into each other) and return the
+// lane's first offset.
+__device__ __forceinline__ uint32_t warp_reserve(uint32_t* ctr, uint32_t mine) {
+  const int lane = threadIdx.x & 31;
+  uint32_t inc = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  uint32_t base = 0u;
+  if (lane == 31 && inc != 0u) base = atomicAdd(ctr, inc);
+  return __shfl_sync(0xFFFFFFFFu, base, 31) + inc - mine;
+}
+
+// Select the kt best keys of a row held by one CTA.
+//   keys[0 … nloc)    order keys of the slice (positions start …), 16-byte
+//                     aligned, key 0 from nloc up to the next multiple of 4
+//   hist1             histogram of keys >> 21 over the visible keys
+//   prepared          the caller ran select_prepare (then a barrier) before the
+//                     scores and counted sm.coarse[0] with select_count_key;
+//                     otherwise this call clears and sums with one barrier
+//   list, list_cap    the production-time list (null: pass A scans the slice);
+//                     list_cap a multiple of 4
+//   cand, cand_cap    scratch for the keys of the level-1 threshold bin
+//                     (cand_cap a multiple of 4)
+//   out               the row's output slots (global memory); positions are
+//                     staged in shared memory when kt ≤ kStage
+// Requires 0 < kt < number of visible keys; all threads of the CTA call it.
+__device__ __forceinline__ void cta_select_row(SelectSmem& sm, const uint32_t* keys, int nloc, int start, int kt,
+                                               const uint32_t* hist1, bool prepared, const uint16_t* list,
+                                               int list_cap, uint16_t* cand, int cand_cap, int32_t* out,
+                                               unsigned long long* tr, const volatile int* abort_flag) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  auto stamp = [&](int slot) {
+    if (tr && tid == 0) tr[slot] = globaltimer_ns();
+  };
+  const bool staged = kt <= kStage;
+  int32_t* const dst = staged ? sm.out_s : out;
+  uint32_t* const hist2 = sm.hist;
+  uint32_t* const hist3 = sm.hist3;
+  uint32_t* const coarse1 = sm.coarse[0];
+  uint32_t* const coarse2 = sm.coarse[1];
+  uint32_t* const coarse3 = sm.coarse[2];
+  if (!prepared) {
+    select_prepare(sm);
+    if (tid < 64) {
+      const uint4* h = reinterpret_cast<const uint4*>(hist1 + 32 * tid);
+      uint32_t s = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 v = h[i];
+        s += v.x + v.y + v.z + v.w;
+      }
+      coarse1[tid] = s;
+    }
+    __syncthreads();
+  }
+  if (abort_flag && *abort_flag) {   // the scores are not valid: the row reads −1
+    for (int i = tid; i < kt; i += nthr) out[i] = -1;
+    return;
+  }
+
+  // ---- level 1 (every warp)
+  int b1, above1;
+  warp_find_bin<kHistBins>(hist1, coarse1, kt, b1, above1);
+  int rem = kt - above1;                      // keys still to take from bin b1 (≥ 1)
+  const int n1 = static_cast<int>(hist1[b1]);
+  const bool done1 = n1 == rem;
+  const bool clist = !done1 && n1 <= cand_cap;   // bin-b1 keys listed; else later passes rescan the slice
+  const uint32_t lo1 = static_cast<uint32_t>(b1) << 21;
+  const int nlist = list ? sm.list_cnt : 0;
+  const bool use_list = list && nlist <= list_cap && lo1 >= sm.filt_lo;
+  stamp(8);
+  if (tr && tid == 0) {
+    tr[9] = use_list ? static_cast<unsigned long long>(nlist) : ~0ull;
+    tr[15] = static_cast<unsigned long long>(n1);
+  }
+
+  // ---- pass A: keys above bin b1 are selected (all of bin b1 too when it
+  // holds exactly the open slots); keys in b1 are listed and histogrammed
+  // done1: keys ≥ lo1 are selected, so no key is both ≤ sel_above and ≥ lo1
+  const uint32_t sel_above = done1 ? lo1 - 1u : lo1 | 0x1FFFFFu;
+  {
+    const PassItems it{keys, use_list ? list : nullptr, use_list ? nlist : (nloc + 3) & ~3};
+    int beg, end;
+    warp_segment(it.n, beg, end);
+    const int lane4 = 4 * (tid & 31);
+    uint32_t cnt = 0;   // selected | candidates << 16
+    for (int i0 = beg + lane4; i0 < end; i0 += 128) {
+      uint32_t kk[4];
+      int ix[4];
+      it.fetch(i0, kk, ix);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) cnt += (kk[u] > sel_above ? 1u : 0u) + (kk[u] >= lo1 ? 0x10000u : 0u);
+    }
+    // the high half counted keys ≥ lo1: keep those inside b1 (none when done1)
+    cnt -= (cnt & 0xFFFFu) << 16;
+    const uint32_t off = warp_reserve(&sm.ctr_gc, cnt);
+    int og = static_cast<int>(off & 0xFFFFu), oc = static_cast<int>(off >> 16);
+    for (int i0 = beg + lane4; i0 < end; i0 += 128) {
+      uint32_t kk[4];
+      int ix[4];
+      it.fetch(i0, kk, ix);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (kk[u] > sel_above) {
+          if (og < kt) dst[og] = start + ix[u];
+          ++og;
+        } else if (kk[u] >= lo1) {
+          if (clist && oc < cand_cap) cand[oc] = static_cast<uint16_t>(ix[u]);
+          ++oc;
+          const uint32_t mid = (kk[u] >> 10) & 0x7FFu;
+          atomicAdd(&hist2[mid], 1u);
+          atomicAdd(&coarse2[mid >> 5], 1u);
+        }
+      }
+    }
+  }
+  __syncthreads();                                                   // barrier 1
+  stamp(10);
+  if (done1) {
+    if (staged)
+      for (int i = tid; i < kt; i += nthr) out[i] = sm.out_s[i];
+    return;
+  }
+  // items of the later passes: the listed keys of bin b1, or the slice filtered by b1
+  const PassItems it{keys, clist ? cand : nullptr, clist ? n1 : (nloc + 3) & ~3};
+  int beg, end;
+  warp_segment(it.n, beg, end);
+  const int lane4 = 4 * (tid & 31);
+
+  // ---- level 2 (every warp) and pass B
+  int b2, above2;
+  warp_find_bin<kHistBins>(hist2, coarse2, rem, b2, above2);
+  rem -= above2;
+  const bool done2 = static_cast<int>(hist2[b2]) == rem;
+  const uint32_t pre22 = static_cast<uint32_t>(b1) << 11 | static_cast<uint32_t>(b2);
+  // selected: the 22-bit prefix above pre22 (or equal when done2) within bin b1
+  const uint32_t sel22 = done2 ? pre22 - 1u : pre22;
+  stamp(11);
+  {
+    uint32_t cnt = 0;
+    for (int i0 = beg + lane4; i0 < end; i0 += 128) {
+      uint32_t kk[4];
+      int ix[4];
+      it.fetch(i0, kk, ix);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t h22 = kk[u] >> 10;
+        cnt += ((h22 >> 11) == static_cast<uint32_t>(b1) && h22 > sel22) ? 1u : 0u;
+      }
+    }
+    int og = static_cast<int>(warp_reserve(&sm.ctr_gc, cnt) & 0xFFFFu);
+    for (int i0 = beg + lane4; i0 < end; i0 += 128) {
+      uint32_t kk[4];
+      int ix[4];
+      it.fetch(i0, kk, ix);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t h22 = kk[u] >> 10;
+        if ((h22 >> 11) != static_cast<uint32_t>(b1)) continue;
+        if (h22 > sel22) {
+          if (og < kt) dst[og] = start + ix[u];
+          ++og;
+        } else if (!done2 && h22 == pre22) {
+          const uint32_t low = kk[u] & 0x3FFu;
+          atomicAdd(&hist3[low], 1u);
+          atomicAdd(&coarse3[low >> 5], 1u);
+        }
+      }
+    }
+  }
+  __syncthreads();                                                   // barrier 2
+  stamp(12);
+  if (!done2) {
+    // ---- level 3 (every warp) and pass C: above the 32-bit threshold, then ties
+    int b3, above3;
+    warp_find_bin<kHistBins / 2>(hist3, coarse3, rem, b3, above3);
+    const int n_gt = kt - rem + above3;       // ties start at this slot
+    rem -= above3;                            // ties to take (≥ 1)
+    const uint32_t thr = pre22 << 10 | static_cast<uint32_t>(b3);
+    stamp(13);
+    uint32_t cnt = 0;
+    for (int i0 = beg + lane4; i0 < end; i0 += 128) {
+      uint32_t kk[4];
+      int ix[4];
+      it.fetch(i0, kk, ix);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if ((kk[u] >> 10) == pre22) cnt += (kk[u] > thr ? 1u : 0u) + (kk[u] == thr ? 0x10000u : 0u);
+    }
+    const uint32_t off = warp_reserve(&sm.ctr_tie, cnt);   // ctr_tie: above | ties << 16, from 0
+    int og = n_gt - above3 + static_cast<int>(off & 0xFFFFu), oe = static_cast<int>(off >> 16);
+    for (int i0 = beg + lane4; i0 < end; i0 += 128) {
+      uint32_t kk[4];
+      int ix[4];
+      it.fetch(i0, kk, ix);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if ((kk[u] >> 10) != pre22) continue;
+        if (kk[u] > thr) {
+          if (og < n_gt) dst[og] = start + ix[u];
+          ++og;
+        } else if (kk[u] == thr) {
+          if (oe < rem) dst[n_gt + oe] = start + ix[u];
+          ++oe;
+        }
+      }
+    }
+    __syncthreads();                                                 // barrier 3
+  }
+  stamp(14);
+  if (staged)
+    for (int i = tid; i < kt; i += nthr) out[i] = sm.out_s[i];
+}
+
+// Select the kt best of a row, one CTA or a cluster.  `cand` is cap ints of
+// scratch: a cluster uses it as its candidate list; one CTA splits it into the
+// production-time list (its first list_cap 16-bit entries; list_cap a multiple
+// of 4, 0 = none) and 16-bit candidate slots.  `prepared`: see cta_select_row.
 __device__ __forceinline__ void cluster_select_row(SelectSmem& sm, const uint32_t* keys, int nloc, int start,
-                                                   int kt, const uint32_t* hist1, int* cand, int cap,
-                                                   int32_t* out, int G, uint32_t rank,
+                                                   int kt, const uint32_t* hist1, int* cand, int cap, int list_cap,
+                                                   bool prepared, int32_t* out, int G, uint32_t rank,
                                                    unsigned long long* tr = nullptr,
                                                    const int* abort_flag = nullptr) {
-  if (G == 1)
-    cluster_select_row_t<false>(sm, keys, nloc, start, kt, hist1, cand, cap, out, G, rank, tr, abort_flag);
-  else
+  if (G == 1) {
+    uint16_t* s16 = reinterpret_cast<uint16_t*>(cand);
+    cta_select_row(sm, keys, nloc, start, kt, hist1, prepared, list_cap > 0 ? s16 : nullptr, list_cap,
+                   s16 + list_cap, (2 * cap - list_cap) & ~3, out, tr, abort_flag);
+  } else {
     cluster_select_row_t<true>(sm, keys, nloc, start, kt, hist1, cand, cap, out, G, rank, tr, abort_flag);
+  }
 }
 
 }  // namespace idx

@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   if (threadIdx.x < 4 && nloc + static_cast<int>(threadIdx.x) < ((nloc + 3) & ~3)) sc_s[nloc + threadIdx.x] = 0u;
   __syncthreads();
   if (tr && threadIdx.x == 0) tr[3] = globaltimer_ns();
-  cluster_select_row(sel, sc_s, nloc, start, kt, hist1, cand, p.cand_cap, out, G, rank, tr);
+  cluster_select_row(sel, sc_s, nloc, start, kt, hist1, cand, p.cand_cap, 0, false, out, G, rank, tr);
   if (rank == 0)
     for (int t = kt + threadIdx.x; t < p.k; t += blockDim.x) out[t] = -1;
   if (G > 1) cluster_sync();
