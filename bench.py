@@ -39,7 +39,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FP8_PER_BF16 = 2.0            # nominal dense fp8 : bf16 tensor ratio on B200
 KEY_BYTES = 128 + 4           # one cached key: 128 e4m3 codes + fp32 scale
 ROW_BYTES_IN = 64 * 128 + 64 * 4   # one query row: 64 heads of e4m3 codes + 64 fp32 weights
-PROFILE_SCORE = os.path.join(ROOT, "profiles", "score_topk_decode_b128_t16384.md")
+PROFILE_SCORE = os.path.join(ROOT, "profiles", "score_decode_b128_t16384.md")
 KERNEL_SOURCES = ["score.cu", "select.cuh", "ptx.cuh"]
 
 
@@ -185,16 +185,19 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     keys, flops, key_rows, score_bytes = workload_numbers(case)
 
-    # the kernel the roofline is about, timed on its own stream with events:
-    # decode — the fused score + top-k; prefill — the tcgen05 scorer writing the
-    # workspace (the step's dominant, tensor-bound kernel), its top-k timed apart
+    # the kernel the roofline is about, timed on its own stream with events: the
+    # tcgen05 scorer writing the workspace when the step uses one (the step's
+    # dominant kernel; its top-k timed apart), else the fused score + top-k
     ws_bytes = X.workspace_size(B, n, max_len, case.k)
+    if ws_bytes:   # the scorer writes fp32 score rows instead of indices
+        score_bytes += B * n * (4 * max_len - 4 * case.k)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
     sc_view = ws.view(torch.float32).view(B, n, max_len) if ws_bytes else None
 
     def score_only():
         if ws_bytes:
-            X.score(q_fp8, w, ix.k_cache, ix.k_scale_cache, lengths, case.causal, max_len, ld=max_len, out=sc_view)
+            X.score_visible(q_fp8, w, ix.k_cache, ix.k_scale_cache, lengths, case.causal, max_len, ld=max_len,
+                            out=sc_view)
         else:
             X.score_topk(q_fp8, w, ix.k_cache, ix.k_scale_cache, lengths, case.causal, case.k, max_len, out=out)
 
@@ -298,9 +301,11 @@ def run_ours(args, rank, world, local_rank):
     ms, score_ms, e2e_ms = max_over_ranks([ms, score_ms, e2e_ms], device=dev)
     if topk_ms is not None:
         topk_ms = max_over_ranks([topk_ms], device=dev)[0]
+    topk_bytes = B * n * 4 * (max_len + case.k) if ws_bytes else None   # score rows read, indices written
     return dict(case=case, keys=keys, flops=flops, key_rows=key_rows, score_bytes=score_bytes, ms=ms,
                 score_ms=score_ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
-                clocks=sampler.summary(), launches=(3 if ws_bytes else 2) * args.steps, topk_ms=topk_ms)
+                clocks=sampler.summary(), launches=(3 if ws_bytes else 2) * args.steps, topk_ms=topk_ms,
+                topk_bytes=topk_bytes, two_pass=bool(ws_bytes))
 
 
 def case_pinned(torch, a):
@@ -449,7 +454,9 @@ def main():
         achieved = r["score_bytes"] / score_s / 1e9
         traffic = profile_traffic(PROFILE_SCORE, r["key_rows"]) if args.workload == DEFAULT_WORKLOAD else None
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": traffic, "peak_source": f"{peak_src} copy bandwidth", "kernel": "score_topk",
+                "traffic": traffic, "peak_source": f"{peak_src} copy bandwidth",
+                "kernel": "score (tcgen05 FP8 scorer, fp32 scores to the workspace)" if r["two_pass"]
+                else "score_topk (fused)",
                 "kernel_us": r["score_ms"] * 1e3, "algorithmic_bytes": r["score_bytes"]}
     line = {
         "metric": metric_name(case), "value": value, "unit": "keys/s", "n_gpus": world, "steps": args.steps,
@@ -470,6 +477,8 @@ def main():
         line["tflops"] = r["flops"] * world / step_s / 1e12      # whole step (quantise + score + top-k)
     if r["topk_ms"] is not None:
         line["topk_us"] = r["topk_ms"] * 1e3
+        line["topk"] = {"us": r["topk_ms"] * 1e3, "algorithmic_bytes": r["topk_bytes"],
+                        "achieved_gbs": r["topk_bytes"] / (r["topk_ms"] / 1e3) / 1e9}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case)
     if rank == 0:

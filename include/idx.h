@@ -142,6 +142,21 @@ IDX_API int idx_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cac
               idx_stream_t stream);
 
 /*
+ * idx_score_visible — the scores of idx_score for the visible keys only, as
+ * the score + top-k path computes them into its workspace: one persistent CTA
+ * per SM, each streaming an equal share of all (row block, 128-key tile)
+ * pairs of the call.
+ *   Arguments as in idx_score, with ld ≥ max_len and w 16-byte aligned.
+ *   scores [B, n, ld]: S for visible keys, −inf from each row's visible count
+ *          up to the end of its last 128-key tile; columns past that tile are
+ *          left unwritten (their contents are unspecified).
+ * Calls with more than 4096 blocks of query rows are served by idx_score.
+ */
+IDX_API int idx_score_visible(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache,
+                              const float* k_scale_cache, const int32_t* lengths, int B, int n, int T_cap,
+                              int max_len, int causal, float* scores, int64_t ld, idx_stream_t stream);
+
+/*
  * idx_topk — Indexer.forward excerpt (top min(index_topk, ·) per row) and the
  * NKI page's output convention (int32, unordered set), on scores already in memory.
  *   scores [B, n, ld] float32 (finite for visible keys); lengths [B]; causal as above.

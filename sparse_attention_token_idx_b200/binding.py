@@ -36,6 +36,7 @@ SIGNATURES = {
     "idx_quant_append": (_I, [_P, _P, _I, _I, _P, _P, _I, _I, _P]),
     "idx_quant_queries_append": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _I, _P, _P, _I, _I, _P]),
     "idx_score": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P]),
+    "idx_score_visible": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P]),
     "idx_topk": (_I, [_P, _P, _I, _I, _I64, _I, _I, _I, _P, _P, _SZ, _P]),
     "idx_score_topk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "idx_score_topk_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
@@ -154,6 +155,23 @@ def score(q_fp8, w, k_cache, k_scale_cache, lengths, causal: bool, max_len: int,
                             _ptr(k_cache, torch.uint8, "k_cache"), _ptr(k_scale_cache, torch.float32, "k_scale"),
                             _ptr(lengths, torch.int32, "lengths"), B, n, T_cap, max_len, int(causal),
                             _ptr(out, torch.float32, "scores"), ld, _stream(stream)), "idx_score")
+    return out
+
+
+def score_visible(q_fp8, w, k_cache, k_scale_cache, lengths, causal: bool, max_len: int, ld: int | None = None,
+                  out=None, stream=None):
+    """Scores [B, n, ld] fp32 of the visible keys (−inf up to the end of each row's
+    last 128-key tile, later columns unwritten): the workspace the score + top-k
+    path fills."""
+    B, n = q_fp8.shape[0], q_fp8.shape[1]
+    T_cap = k_cache.shape[1]
+    ld = ld if ld is not None else max_len
+    out = out if out is not None else torch.empty((B, n, ld), dtype=torch.float32, device=q_fp8.device)
+    _check(load().idx_score_visible(_ptr(q_fp8, torch.uint8, "q_fp8"), _ptr(w, torch.float32, "w"),
+                                    _ptr(k_cache, torch.uint8, "k_cache"),
+                                    _ptr(k_scale_cache, torch.float32, "k_scale"),
+                                    _ptr(lengths, torch.int32, "lengths"), B, n, T_cap, max_len, int(causal),
+                                    _ptr(out, torch.float32, "scores"), ld, _stream(stream)), "idx_score_visible")
     return out
 
 

@@ -189,9 +189,13 @@ extern "C" const char* idx_error_string(int code) {
 extern "C" size_t idx_workspace_size(int B, int n, int max_len, int k) {
   (void)k;
   if (B <= 0 || n <= 0 || max_len <= 0) return 0;
-  if (n <= 2) return 0;   // decode-shaped calls select in shared memory
-  // prefill-shaped calls: one fp32 score row of max_len columns per query row
-  return static_cast<size_t>(B) * static_cast<size_t>(n) * static_cast<size_t>(max_len) * sizeof(float);
+  // Decode-shaped calls select in shared memory (fused score + top-k): their
+  // cache stream is HBM-bound either way, and the fused kernel skips the
+  // score round trip and the second launch.
+  const int64_t rows = static_cast<int64_t>(B) * n;
+  if (n <= 2) return 0;
+  // one fp32 score row of max_len columns per query row
+  return static_cast<size_t>(rows) * static_cast<size_t>(max_len) * sizeof(float);
 }
 
 extern "C" void idx_debug_set(unsigned int flags, unsigned long long budget_ns) {

@@ -26,6 +26,14 @@ bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64
 
 unsigned long long* trace_buffer();  // device address of the phase-trace buffer
 
+// Flat-partition scorer (flat_score.cu): scores of every visible (row, key) of
+// the call into scores [B, n, ld], one persistent CTA per SM; columns past a
+// row's last key tile are left unwritten.  IDX_ERR_UNSUPPORTED when the call
+// has more row blocks than the kernel's shared-memory index holds.
+int launch_flat_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
+                      const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, float* scores,
+                      int64_t ld, cudaStream_t stream);
+
 struct DebugState {
   unsigned int flags;
   unsigned long long budget_ns;

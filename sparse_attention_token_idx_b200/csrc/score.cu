@@ -70,16 +70,24 @@ struct Cfg {
   static constexpr int kTokPerWarp = NT / kTokGroups;
   static constexpr int kWarpsPerTile = EPI_WARPS / TSPLIT;   // warps that consume one tile
   static constexpr int kQBytes = N * IDX_DIM;
-  static constexpr int kCand = NT == 1 ? 4096 : 1024;     // scratch ints of the select
+  static constexpr int kCand = NT == 1 ? 3584 : 1024;     // scratch ints of the select
   // one row per CTA: 16-bit entries of the scratch that hold the production-time list
-  static constexpr int kList = (FUSED && NT == 1) ? 6144 : 0;
+  static constexpr int kList = (FUSED && NT == 1) ? 5120 : 0;
+  // key scales sit in their own ring, freed by the epilogue, so that a key stage
+  // is freed as soon as the MMA has read it: producer ≤ STAGES tiles ahead of the
+  // MMA, the MMA ≤ NUM_ACC ahead of the epilogue
+  static constexpr int kScaleSlots = 2 * STAGES;
+  static_assert(kScaleSlots >= STAGES + NUM_ACC, "scale ring");
+  // unfused one-row CTAs are small work items: two share an SM (register budget
+  // 65536 / (2 × threads)), so one CTA's set-up and drain overlap the other's stream
+  static constexpr int kMinCtas = (!FUSED && NT == 1) ? 2 : 1;
   // shared memory carve (offsets from a 1024-aligned base)
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffScale = kOffK + STAGES * kTileBytes;
-  static constexpr int kOffW = kOffScale + STAGES * kTileKeys * 4;
+  static constexpr int kOffW = kOffScale + kScaleSlots * kTileKeys * 4;
   static constexpr int kOffBar = kOffW + N * 4;
-  static constexpr int kNumBars = 2 * STAGES + 2 * NUM_ACC + 3;
+  static constexpr int kNumBars = 2 * STAGES + kScaleSlots + 2 * NUM_ACC + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffSel = (kOffMisc + 64 + 127) / 128 * 128;
   static constexpr int kOffHist1 = kOffSel + (FUSED ? static_cast<int>(sizeof(SelectSmem)) : 0);
@@ -93,7 +101,8 @@ struct Cfg {
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT, bool W_REGS>
-__global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>::kThreads, 1)
+__global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>::kThreads,
+                                  Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>::kMinCtas)
     score_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                  const __grid_constant__ CUtensorMap tmap_s, const ScoreParams p) {
   using C = Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>;
@@ -108,7 +117,8 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
-  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* sc_empty = bars + 2 * STAGES;   // [C::kScaleSlots]
+  uint64_t* acc_full = sc_empty + C::kScaleSlots;
   uint64_t* acc_empty = acc_full + NUM_ACC;
   uint64_t* q_full = acc_empty + NUM_ACC;
   uint64_t* drain_bar = q_full + 1;
@@ -131,7 +141,9 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
     tr[0] = globaltimer_ns();
     tr[7] = smid;
   }
-  const uint32_t rank = cluster_rank();
+  // fused calls split a row over a cluster (the selection exchanges through
+  // distributed shared memory); unfused calls split it over plain CTAs
+  const uint32_t rank = FUSED ? cluster_rank() : static_cast<uint32_t>(blockIdx.x % p.G);
   const int G = p.G;
   const int item = blockIdx.x / G;
   const int b = item % p.B;
@@ -161,8 +173,9 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + C::kWarpsPerTile);   // MMA done with the keys, epilogue with the scales
+      mbar_init(&empty[s], 1);   // the MMA is done with the keys
     }
+    for (int c = 0; c < C::kScaleSlots; ++c) mbar_init(&sc_empty[c], C::kWarpsPerTile);   // epilogue done with the scales
     for (int a = 0; a < NUM_ACC; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], C::kWarpsPerTile);
@@ -171,7 +184,7 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
     mbar_init(drain_bar, 1);
     mbar_init(never_bar, 1);
     *abort_flag = 0;
-    if constexpr (FUSED) row_filter_reset(sel);
+    if constexpr (FUSED) row_filter_reset(sel.cta);
     fence_barrier_init();
     // Thread 0 is also the TMA producer: start the query and the first STAGES
     // key tiles now, so that their DRAM latency overlaps the rest of the set-up
@@ -201,7 +214,7 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
   }
   if constexpr (FUSED) {
     for (int i = threadIdx.x; i < NT * kHistBins; i += blockDim.x) hist1[i] = 0;
-    if constexpr (NT == 1) select_prepare(sel);   // one row: the selection state is set up here
+    if constexpr (NT == 1) select_prepare(sel.cta);   // one row: the selection state is set up here
   }
   tc_fence_before();
   __syncthreads();
@@ -217,11 +230,13 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
       int t = tma_issued;   // the first tiles went out during set-up
       for (; t < ntiles; ++t) {
         const int s = t % STAGES;
+        const int c = t % C::kScaleSlots;
         if (!mbar_wait(&empty[s], ((t / STAGES) & 1) ^ 1, budget, abort_flag, p.err)) break;
+        if (!mbar_wait(&sc_empty[c], ((t / C::kScaleSlots) & 1) ^ 1, budget, abort_flag, p.err)) break;
         mbar_arrive_expect_tx(&full[s], kTileBytes + kTileKeys * 4);
         const int tt = tile_of(t);
         tma_load_3d(k_s + s * kTileBytes, &tmap_k, &full[s], 0, start + tt * kTileKeys, b);
-        tma_load_2d(scale_s + s * kTileKeys, &tmap_s, &full[s], start + tt * kTileKeys, b);
+        tma_load_2d(scale_s + c * kTileKeys, &tmap_s, &full[s], start + tt * kTileKeys, b);
       }
       tma_issued = t;
     }
@@ -276,13 +291,14 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
       const int s = t % STAGES;
       const int tt = tile_of(t);
       const int key = start + tt * kTileKeys + kl;
+      const int sc_slot = t % C::kScaleSlots;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&acc_full[a], (t / NUM_ACC) & 1, budget, abort_flag, p.err) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       if (trace && t == 0 && ew == 0 && lane == 0) tr[2] = globaltimer_ns();
       tc_fence_after();
-      const float ks = scale_s[s * kTileKeys + kl];   // landed with the keys (same barrier)
+      const float ks = scale_s[sc_slot * kTileKeys + kl];   // landed with the keys (same barrier)
 #pragma unroll
       for (int jj = 0; jj < C::kTokPerWarp; ++jj) {
         const int j = tok_lo + jj;
@@ -330,12 +346,12 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
           const uint32_t u = order_key(sc);
           sc_s[j * p.chunk_cap + tt * kTileKeys + kl] = visible ? u : 0u;
           if (visible) {
-            if constexpr (NT == 1) select_count_key(sel, hist1, u);   // with the coarse sums
+            if constexpr (NT == 1) select_count_key(sel.cta, hist1, u);   // with the coarse sums
             else atomicAdd(&hist1[j * kHistBins + (u >> 21)], 1u);
           }
           // one row per CTA: keys that may reach the top k go to the short list
           if constexpr (C::kList > 0)
-            if (G == 1) row_filter_append(sel, list16, C::kList, u, visible, tt * kTileKeys + kl);
+            if (G == 1) row_filter_append(sel.cta, list16, C::kList, u, visible, tt * kTileKeys + kl);
         } else {
           if (row_exists(j) && key < p.ld) {
             p.scores[(static_cast<int64_t>(b) * p.n + row0 + j) * p.ld + key] = visible ? sc : -INFINITY;
@@ -346,14 +362,14 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&acc_empty[a]);
-        mbar_arrive(&empty[s]);
+        mbar_arrive(&sc_empty[sc_slot]);
       }
       // the first epilogue warp raises the list's bound after tile 4 and every 8 tiles
       if constexpr (C::kList > 0) {
         if (G == 1 && ew == 0 && (t == 4 || (t >= 8 && (t & 7) == 0))) {
           const int v0 = row_vis(0);
           const int target = row_filter_target((t + 1) * kTileKeys, v0, min(p.k, v0));
-          if (target > 0) row_filter_raise(sel, hist1, target);
+          if (target > 0) row_filter_raise(sel.cta, hist1, target);
         }
       }
     }
@@ -452,21 +468,36 @@ int launch_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, c
   const int ntb = (n + NT - 1) / NT;
   const int64_t items = static_cast<int64_t>(B) * ntb;
   const int sms = num_sms();
-  // cluster size: enough CTAs to cover the GPU once, and (fused) a score slice that fits
-  int G = 1;
-  if (items < sms) G = pow2_floor(static_cast<int>(sms / items));
-  G = G > 8 ? 8 : G;
-  const int min_keys_per_cta = 512;
-  while (G > 1 && (max_len + G - 1) / G < min_keys_per_cta) G /= 2;
   auto chunk_of = [&](int g) { return ((max_len + g - 1) / g + kTileKeys - 1) / kTileKeys * kTileKeys; };
-  if (FUSED)
-    while (G < 8 && NT * chunk_of(G) * 4 > score_budget_bytes) G *= 2;
-  const int chunk_cap = chunk_of(G);
-  int smem = C::smem_bytes(FUSED ? chunk_cap : 0);
-  // TMEM has 512 columns per SM and tcgen05.alloc waits for free columns: size the
-  // shared-memory request so that co-resident CTAs never ask for more than 512 in total
+  // TMEM has 512 columns per SM and tcgen05.alloc waits for free columns: the
+  // shared-memory request keeps co-resident CTAs within 512 columns in total
   const int tmem_ctas = 512 / C::kTmemCols;
   const int per_sm = smem_per_sm();
+  const int min_keys_per_cta = 512;
+  int G = 1;
+  if (FUSED) {
+    // cluster size: enough CTAs to cover the GPU once, and a score slice that fits
+    if (items < sms) G = pow2_floor(static_cast<int>(sms / items));
+    G = G > 8 ? 8 : G;
+    while (G > 1 && (max_len + G - 1) / G < min_keys_per_cta) G /= 2;
+    while (G < 8 && NT * chunk_of(G) * 4 > score_budget_bytes) G *= 2;
+  } else if (items < 4 * static_cast<int64_t>(sms)) {
+    // rows split over plain CTAs: the split whose busiest SM streams the fewest
+    // keys (CTAs spread evenly over the SMs), with a fixed cost per CTA
+    int64_t best = -1;
+    for (int g = 1; g <= 16; g *= 2) {
+      if (g > 1 && (max_len + g - 1) / g < min_keys_per_cta) break;
+      const int64_t ctas = items * g;
+      const int64_t per_sm_ctas = (ctas + sms - 1) / sms;
+      const int64_t cost = per_sm_ctas * (chunk_of(g) + 128);
+      if (best < 0 || cost < best) {
+        best = cost;
+        G = g;
+      }
+    }
+  }
+  const int chunk_cap = chunk_of(G);
+  int smem = C::smem_bytes(FUSED ? chunk_cap : 0);
   while (per_sm / (smem + 1024) > tmem_ctas) smem += 1024;
   if (smem > max_dynamic_smem()) return IDX_ERR_SHAPE;
   if (items * G > 0x7FFFFFFF) return IDX_ERR_SHAPE;
@@ -515,7 +546,7 @@ int launch_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, c
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(G);
+  attr[0].val.clusterDim.x = static_cast<unsigned>(FUSED ? G : 1);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
@@ -558,10 +589,24 @@ extern "C" int idx_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_
   if (ld <= 0) return IDX_ERR_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (n <= kDecodeRowsMax)
-    return launch_score<1, false, 6, 4, 8, 2, true>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
-                                           scores, ld, 0, nullptr, s, 0);
+    return launch_score<1, false, 4, 4, 8, 2, false>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len,
+                                            causal, scores, ld, 0, nullptr, s, 0);
   return launch_score<4, false, 4, 2, 16, 1, false>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
                                          scores, ld, 0, nullptr, s, 0);
+}
+
+extern "C" int idx_score_visible(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache,
+                                 const float* k_scale_cache, const int32_t* lengths, int B, int n, int T_cap,
+                                 int max_len, int causal, float* scores, int64_t ld, idx_stream_t stream) {
+  const int c = check_score_args(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal);
+  if (c <= 0) return c;
+  if (!scores) return IDX_ERR_NULL;
+  if (ld < max_len) return IDX_ERR_SHAPE;
+  // flat partition over every SM when the call fits its index, else per row block
+  const int r = launch_flat_score(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal, scores,
+                                  ld, reinterpret_cast<cudaStream_t>(stream));
+  if (r != IDX_ERR_UNSUPPORTED) return r;
+  return idx_score(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal, scores, ld, stream);
 }
 
 extern "C" int idx_score_topk(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache,
@@ -577,12 +622,14 @@ extern "C" int idx_score_topk(const uint8_t* q_fp8, const float* w, const uint8_
   // (the tcgen05 scorer at full tensor throughput), then the top-k kernel with
   // several rows per SM in flight.  A row's selection then overlaps other rows'
   // work instead of stalling its CTA's MMA pipeline.
+  // Decode-shaped calls with many rows take the same route: the scorer then
+  // splits rows over every SM instead of holding one row per CTA.
   const size_t need = idx_workspace_size(B, n, max_len, k);
-  if (n > kDecodeRowsMax && ws && ws_bytes >= need && need > 0) {
+  if (ws && ws_bytes >= need && need > 0) {
     if (reinterpret_cast<uintptr_t>(ws) & 15) return IDX_ERR_ALIGN;
     float* scores = static_cast<float*>(ws);
-    const int r = launch_score<4, false, 4, 2, 16, 1, false>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap,
-                                                             max_len, causal, scores, max_len, 0, nullptr, s, 0);
+    const int r = idx_score_visible(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal, scores,
+                                    max_len, stream);
     if (r != IDX_OK) return r;
     return idx_topk(scores, lengths, B, n, max_len, max_len, causal, k, indices, nullptr, 0, stream);
   }

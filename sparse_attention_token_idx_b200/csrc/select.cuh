@@ -43,9 +43,19 @@ struct Grp {
   }
 };
 
+// State of the one-CTA selection (cta_select_row) and of the row filter.
+struct alignas(16) CtaSelSmem {
+  uint32_t hist[kHistBins];      // level-2 histogram
+  uint32_t hist3[kHistBins / 2]; // level-3 histogram (own buffer: one barrier per exchange)
+  uint32_t coarse[3][64];        // coarse sums (32 fine bins per entry) of levels 1-3
+  uint32_t ctr_gc;               // output slots taken (low 16 bits) | bin-b1 keys listed (high)
+  uint32_t ctr_tie;              // above the 32-bit threshold (low) | ties seen (high)
+  uint32_t filt_lo;              // row filter: keys below this bound are not listed
+  int list_cnt;                  // row filter: list entries taken
+};
+
 struct alignas(16) SelectSmem {
-  uint32_t hist[kHistBins];      // this CTA's level-2 histogram
-  uint32_t hist3[kHistBins / 2]; // this CTA's level-3 histogram (own buffer: one barrier per exchange)
+  CtaSelSmem cta;                // one-CTA path; its hist / hist3 are also the cluster path's
   uint32_t hsum[kHistBins];      // cluster-summed histogram
   int warp_a[32];
   int warp_b[32];
@@ -55,11 +65,6 @@ struct alignas(16) SelectSmem {
   int cta_base[2];               // cluster prefix of those totals for this CTA
   int any_abort;
   int pad[3];
-  uint32_t coarse[3][64];        // one-CTA path: coarse histograms (32 fine bins per entry) of levels 1-3
-  uint32_t ctr_gc;               // one-CTA path: output slots taken (low 16 bits) | bin-b1 keys listed (high)
-  uint32_t ctr_tie;              // one-CTA path: ties at the 32-bit threshold seen
-  uint32_t filt_lo;              // row filter: keys below this bound are not listed
-  int list_cnt;                  // row filter: list entries taken
   int32_t out_s[kStage];         // staged positions of the current row (CTA 0's copy is the one used)
 };
 
@@ -265,8 +270,8 @@ __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint3
   ro.staged = kt <= kStage;
   ro.stage_local = sm.out_s;
   ro.stage_base = CL ? dsmem_addr(sm.out_s, 0) : 0u;
-  for (int i = tid; i < kHistBins; i += nthr) sm.hist[i] = 0;
-  for (int i = tid; i < kHistBins / 2; i += nthr) sm.hist3[i] = 0;
+  for (int i = tid; i < kHistBins; i += nthr) sm.cta.hist[i] = 0;
+  for (int i = tid; i < kHistBins / 2; i += nthr) sm.cta.hist3[i] = 0;
 
   // ---- level 1
   const uint32_t* H = summed_hist<CL>(sm, hist1, kHistBins, G, rank, abort_flag);
@@ -333,21 +338,21 @@ __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint3
   __syncthreads();
   // ---- level-2 histogram over the candidates (or the whole slice on overflow)
   if (!overflow) {
-    for (int c = tid; c < te; c += nthr) atomicAdd(&sm.hist[(keys[cand[c]] >> 10) & 0x7FF], 1u);
+    for (int c = tid; c < te; c += nthr) atomicAdd(&sm.cta.hist[(keys[cand[c]] >> 10) & 0x7FF], 1u);
   } else {
     for (int i = tid; i < nloc; i += nthr) {
       const uint32_t key = keys[i];
-      if ((key >> 21) == b1) atomicAdd(&sm.hist[(key >> 10) & 0x7FF], 1u);
+      if ((key >> 21) == b1) atomicAdd(&sm.cta.hist[(key >> 10) & 0x7FF], 1u);
     }
   }
   stamp(11);
   // ---- level 2
-  const uint32_t* H2 = summed_hist<CL>(sm, sm.hist, kHistBins, G, rank);
+  const uint32_t* H2 = summed_hist<CL>(sm, sm.cta.hist, kHistBins, G, rank);
   find_bin(sm, H2, kHistBins, rem);
   const uint32_t b2 = static_cast<uint32_t>(sm.bin);
   rem -= sm.above;
   const bool done2 = static_cast<int>(H2[b2]) == rem;
-  __syncthreads();                           // everyone has read H2 (it may be sm.hist)
+  __syncthreads();                           // everyone has read H2 (it may be sm.cta.hist)
   // ---- pass B: over the candidates
   const int trips_b = (nscan + nthr - 1) / nthr;
   cg = 0;
@@ -359,7 +364,7 @@ __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint3
         const uint32_t mid = (key >> 10) & 0x7FF;
         const bool eq = mid == b2;
         cg += (mid > b2 || (done2 && eq)) ? 1 : 0;
-        if (!done2 && eq) atomicAdd(&sm.hist3[key & 0x3FF], 1u);
+        if (!done2 && eq) atomicAdd(&sm.cta.hist3[key & 0x3FF], 1u);
       }
     }
   }
@@ -387,7 +392,7 @@ __device__ __forceinline__ void cluster_select_row_t(SelectSmem& sm, const uint3
   }
   stamp(13);
   // ---- level 3
-  const uint32_t* H3 = summed_hist<CL>(sm, sm.hist3, 1024, G, rank);
+  const uint32_t* H3 = summed_hist<CL>(sm, sm.cta.hist3, 1024, G, rank);
   find_bin(sm, H3, 1024, rem);
   const uint32_t b3 = static_cast<uint32_t>(sm.bin);
   const int above3 = sm.above;
@@ -469,7 +474,7 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 
 // Zero the level-2/3 histograms, their coarse sums, the level-1 coarse sums
 // and the pass counters (block-wide; a barrier must follow before use).
-__device__ __forceinline__ void select_prepare(SelectSmem& sm) {
+__device__ __forceinline__ void select_prepare(CtaSelSmem& sm) {
   const int tid = threadIdx.x, nthr = blockDim.x;
   for (int i = tid; i < kHistBins / 4; i += nthr) reinterpret_cast<uint4*>(sm.hist)[i] = make_uint4(0u, 0u, 0u, 0u);
   for (int i = tid; i < kHistBins / 8; i += nthr) reinterpret_cast<uint4*>(sm.hist3)[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -531,7 +536,7 @@ __device__ __forceinline__ void warp_find_bin(const uint32_t* hist, const uint32
 }
 
 // Production side, per key: level-1 histogram and its coarse sums.
-__device__ __forceinline__ void select_count_key(SelectSmem& sm, uint32_t* hist1, uint32_t key) {
+__device__ __forceinline__ void select_count_key(CtaSelSmem& sm, uint32_t* hist1, uint32_t key) {
   atomicAdd(&hist1[key >> 21], 1u);
   atomicAdd(&sm.coarse[0][key >> 26], 1u);
 }
@@ -540,7 +545,7 @@ __device__ __forceinline__ void select_count_key(SelectSmem& sm, uint32_t* hist1
 // its own key): visible keys at or above the current bound are appended to the
 // list at slice index idx.  Entries past the capacity are dropped (the count
 // still grows, which marks the list incomplete).
-__device__ __forceinline__ void row_filter_append(SelectSmem& sm, uint16_t* list, int cap, uint32_t key,
+__device__ __forceinline__ void row_filter_append(CtaSelSmem& sm, uint16_t* list, int cap, uint32_t key,
                                                   bool visible, int idx) {
   const uint32_t lo = *reinterpret_cast<const volatile uint32_t*>(&sm.filt_lo);
   const bool p = visible && key >= lo;
@@ -553,11 +558,67 @@ __device__ __forceinline__ void row_filter_append(SelectSmem& sm, uint16_t* list
   if (p && pos < cap) list[pos] = static_cast<uint16_t>(idx);
 }
 
+// As row_filter_append, with the caller's own test (`take`, visible and at or
+// above a bound it read once).
+__device__ __forceinline__ void row_filter_append_at(CtaSelSmem& sm, uint16_t* list, int cap, uint32_t key,
+                                                     bool take, int idx) {
+  (void)key;
+  const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
+  if (m == 0u) return;
+  int base = 0;
+  if ((threadIdx.x & 31) == 0) base = atomicAdd(&sm.list_cnt, __popc(m));
+  base = __shfl_sync(0xFFFFFFFFu, base, 0);
+  const int pos = base + __popc(m & lanemask_lt());
+  if (take && pos < cap) list[pos] = static_cast<uint16_t>(idx);
+}
+
+// As row_filter_raise, for producers that count only the fine histogram: each
+// lane sums 64 bins, then the lane's 64 bins are resolved in pairs.
+__device__ __forceinline__ void row_filter_raise_fine(CtaSelSmem& sm, const uint32_t* hist1, int target) {
+  const int lane = threadIdx.x & 31;
+  // lane l sums bins 1984 − 64l … 2047 − 64l (descending over the lanes)
+  const uint4* h4 = reinterpret_cast<const uint4*>(hist1 + 1984 - 64 * lane);
+  int s = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint4 v = h4[i];
+    s += static_cast<int>(v.x + v.y + v.z + v.w);
+  }
+  int inc = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  const uint32_t hit = __ballot_sync(0xFFFFFFFFu, inc >= target);
+  if (hit == 0u) return;
+  const int L = __ffs(hit) - 1;
+  const int exc_l = __shfl_sync(0xFFFFFFFFu, inc - s, L);
+  const int hi = 2047 - 64 * L;             // lane j takes bins hi − 2j (higher) and hi − 2j − 1
+  const uint2 pr = *reinterpret_cast<const uint2*>(hist1 + hi - 2 * lane - 1);
+  const int a = static_cast<int>(pr.y), b = static_cast<int>(pr.x);
+  int inc2 = a + b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xFFFFFFFFu, inc2, o);
+    if (lane >= o) inc2 += t;
+  }
+  const uint32_t hit2 = __ballot_sync(0xFFFFFFFFu, exc_l + inc2 >= target);
+  const int J = hit2 ? __ffs(hit2) - 1 : 31;
+  const int exc2 = __shfl_sync(0xFFFFFFFFu, inc2 - a - b, J);
+  const int aJ = __shfl_sync(0xFFFFFFFFu, a, J);
+  const int bin = exc_l + exc2 + aJ >= target ? hi - 2 * J : hi - 2 * J - 1;
+  if (lane == 0) {
+    const uint32_t lo = static_cast<uint32_t>(bin) << 21;
+    if (lo > sm.filt_lo) sm.filt_lo = lo;
+  }
+}
+
 // Raise the bound, one warp (warp-collective): the highest bin L such that at
 // least `target` of the keys counted so far lie in bins ≥ L.  Other warps may
 // still be adding to the histograms; every count read is at most its final
 // value, so L never exceeds what the keys seen so far support.
-__device__ __forceinline__ void row_filter_raise(SelectSmem& sm, const uint32_t* hist1, int target) {
+__device__ __forceinline__ void row_filter_raise(CtaSelSmem& sm, const uint32_t* hist1, int target) {
   int bin, above;
   warp_find_bin<kHistBins>(hist1, sm.coarse[0], target, bin, above);
   // a miss (fewer than target keys counted) or a racy read leaves bin 0: no raise
@@ -576,7 +637,7 @@ __device__ __forceinline__ int row_filter_target(int m, int vis, int kt) {
 }
 
 // Reset the row filter (one thread; a barrier must follow before production).
-__device__ __forceinline__ void row_filter_reset(SelectSmem& sm) {
+__device__ __forceinline__ void row_filter_reset(CtaSelSmem& sm) {
   sm.filt_lo = 0u;
   sm.list_cnt = 0;
 }
@@ -643,19 +704,22 @@ __device__ __forceinline__ uint32_t warp_reserve(uint32_t* ctr, uint32_t mine) {
 //                     list_cap a multiple of 4
 //   cand, cand_cap    scratch for the keys of the level-1 threshold bin
 //                     (cand_cap a multiple of 4)
-//   out               the row's output slots (global memory); positions are
-//                     staged in shared memory when kt ≤ kStage
+//   out               the row's output slots (global memory)
+//   stage             shared memory for kStage positions, or null: when given
+//                     and kt ≤ kStage, positions are staged there and written
+//                     to `out` with coalesced stores at the end
 // Requires 0 < kt < number of visible keys; all threads of the CTA call it.
-__device__ __forceinline__ void cta_select_row(SelectSmem& sm, const uint32_t* keys, int nloc, int start, int kt,
+__device__ __forceinline__ void cta_select_row(CtaSelSmem& sm, const uint32_t* keys, int nloc, int start, int kt,
                                                const uint32_t* hist1, bool prepared, const uint16_t* list,
                                                int list_cap, uint16_t* cand, int cand_cap, int32_t* out,
-                                               unsigned long long* tr, const volatile int* abort_flag) {
+                                               int32_t* stage, unsigned long long* tr,
+                                               const volatile int* abort_flag) {
   const int tid = threadIdx.x, nthr = blockDim.x;
   auto stamp = [&](int slot) {
     if (tr && tid == 0) tr[slot] = globaltimer_ns();
   };
-  const bool staged = kt <= kStage;
-  int32_t* const dst = staged ? sm.out_s : out;
+  const bool staged = stage && kt <= kStage;
+  int32_t* const dst = staged ? stage : out;
   uint32_t* const hist2 = sm.hist;
   uint32_t* const hist3 = sm.hist3;
   uint32_t* const coarse1 = sm.coarse[0];
@@ -740,7 +804,7 @@ __device__ __forceinline__ void cta_select_row(SelectSmem& sm, const uint32_t* k
   stamp(10);
   if (done1) {
     if (staged)
-      for (int i = tid; i < kt; i += nthr) out[i] = sm.out_s[i];
+      for (int i = tid; i < kt; i += nthr) out[i] = stage[i];
     return;
   }
   // items of the later passes: the listed keys of bin b1, or the slice filtered by b1
@@ -831,7 +895,7 @@ __device__ __forceinline__ void cta_select_row(SelectSmem& sm, const uint32_t* k
   }
   stamp(14);
   if (staged)
-    for (int i = tid; i < kt; i += nthr) out[i] = sm.out_s[i];
+    for (int i = tid; i < kt; i += nthr) out[i] = stage[i];
 }
 
 // Select the kt best of a row, one CTA or a cluster.  `cand` is cap ints of
@@ -845,8 +909,8 @@ __device__ __forceinline__ void cluster_select_row(SelectSmem& sm, const uint32_
                                                    const int* abort_flag = nullptr) {
   if (G == 1) {
     uint16_t* s16 = reinterpret_cast<uint16_t*>(cand);
-    cta_select_row(sm, keys, nloc, start, kt, hist1, prepared, list_cap > 0 ? s16 : nullptr, list_cap,
-                   s16 + list_cap, (2 * cap - list_cap) & ~3, out, tr, abort_flag);
+    cta_select_row(sm.cta, keys, nloc, start, kt, hist1, prepared, list_cap > 0 ? s16 : nullptr, list_cap,
+                   s16 + list_cap, (2 * cap - list_cap) & ~3, out, sm.out_s, tr, abort_flag);
   } else {
     cluster_select_row_t<true>(sm, keys, nloc, start, kt, hist1, cand, cap, out, G, rank, tr, abort_flag);
   }

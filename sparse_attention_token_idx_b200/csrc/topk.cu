@@ -103,6 +103,201 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const TopkParams 
   if (tr && threadIdx.x == 0) tr[4] = globaltimer_ns();
 }
 
+// ---------------------------------------------------------------------------
+// Rows held by one CTA.  The visible scores arrive by 1-D bulk copies of 16 KB,
+// all issued at once; as each lands, a pass over shared memory turns it into
+// order keys, counts the level-1 histogram and its coarse sums, and keeps the
+// short list of keys that may reach the top k (row_filter_*); then
+// cta_select_row writes the positions straight to global memory.  Several
+// CTAs share an SM, so one row's selection overlaps another's copies.
+
+constexpr int kRowThreads = 512;    // one-CTA rows longer than 8192 keys: 16 warps
+constexpr int kRowChunk = 4096;     // floats per bulk copy
+constexpr int kRowMaxChunks = 4;    // rows of up to 16384 keys
+
+struct RowLayout {
+  int hist1, scratch, keys, bars, total;
+};
+
+__host__ __device__ inline RowLayout row_layout(int chunk_cap, int list_cap, int cand_cap) {
+  RowLayout l;
+  l.hist1 = (static_cast<int>(sizeof(CtaSelSmem)) + 127) / 128 * 128;
+  l.scratch = l.hist1 + kHistBins * 4;
+  l.keys = l.scratch + ((list_cap + cand_cap) * 2 + 15) / 16 * 16;
+  l.bars = l.keys + chunk_cap * 4;
+  l.total = l.bars + kRowMaxChunks * 8;
+  return l;
+}
+
+struct RowParams {
+  const float* scores;
+  const int32_t* lengths;
+  int32_t* indices;
+  int64_t ld;
+  int B, n, max_len, causal, k;
+  int chunk_cap, list_cap, cand_cap;
+  unsigned long long budget_ns;
+  unsigned int* err;
+  unsigned long long* trace;
+};
+
+__global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(const RowParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);   // shared-space pointer
+  const RowLayout L = row_layout(p.chunk_cap, p.list_cap, p.cand_cap);
+  CtaSelSmem& sel = *reinterpret_cast<CtaSelSmem*>(smem);
+  uint32_t* hist1 = reinterpret_cast<uint32_t*>(smem + L.hist1);
+  uint16_t* list16 = reinterpret_cast<uint16_t*>(smem + L.scratch);
+  uint16_t* cand16 = list16 + p.list_cap;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L.keys);   // fp32 scores until converted
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  __shared__ int timed_out;
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  unsigned long long* tr = (p.trace && blockIdx.x < 8192) ? p.trace + blockIdx.x * kTraceSlotsT : nullptr;
+  if (tr && tid == 0) tr[0] = globaltimer_ns();
+  const int64_t row = blockIdx.x;              // b * n + i
+  const int b = static_cast<int>(row / p.n);
+  const int i = static_cast<int>(row - static_cast<int64_t>(b) * p.n);
+  const int len = p.lengths[b];
+  const bool bad = len < p.n || len > p.max_len;
+  if (bad && tid == 0 && i == 0) raise_error(p.err, IDX_DEV_ERR_LENGTH);
+  const int vis = bad ? 0 : (p.causal ? len - p.n + i + 1 : len);
+  int32_t* out = p.indices + row * p.k;
+  const int kt = min(p.k, vis);
+  if (kt == vis) {   // every visible position is selected (or none is visible)
+    for (int t = tid; t < p.k; t += nthr) out[t] = t < kt ? t : -1;
+    return;
+  }
+  const float* src = p.scores + row * p.ld;
+  const int n4 = (vis + 3) & ~3;               // floats copied: within the row, since ld % 4 == 0
+  const int nchunks = (n4 + kRowChunk - 1) / kRowChunk;
+  if (tid == 0) {
+    for (int c = 0; c < nchunks; ++c) mbar_init(&bars[c], 1);
+    fence_barrier_init();
+    for (int c = 0; c < nchunks; ++c) {
+      const int cnt = min(kRowChunk, n4 - c * kRowChunk);
+      mbar_arrive_expect_tx(&bars[c], static_cast<uint32_t>(cnt) * 4u);
+      bulk_load(keys + c * kRowChunk, src + c * kRowChunk, static_cast<uint32_t>(cnt) * 4u, &bars[c]);
+    }
+    row_filter_reset(sel);
+    timed_out = 0;
+  }
+  select_prepare(sel);
+  for (int t = tid; t < kHistBins; t += nthr) hist1[t] = 0u;
+  __syncthreads();
+  // the list pays off when the k best are a small share of the row
+  const bool use_list = p.list_cap > 0 && vis >= 4 * kt;
+  const int warp = tid >> 5;
+  // floats [lo, hi) → order keys in place (key 0 past vis), counted in the
+  // level-1 histogram; with `list`, keys at or above the bound go to the list
+  // (one shared atomic per warp and 128 keys).  Trip count uniform per warp.
+  const uint32_t lt = lanemask_lt();
+  auto convert = [&](int lo, int hi, bool list, bool keys_ready) {
+    const uint32_t bound = *reinterpret_cast<const volatile uint32_t*>(&sel.filt_lo);
+    for (int base = lo; base < hi; base += 4 * nthr) {
+      const int i0 = base + 4 * tid;
+      uint32_t u[4] = {0u, 0u, 0u, 0u};
+      if (i0 < hi) {
+        const uint4 v = *reinterpret_cast<const uint4*>(keys + i0);
+        const uint32_t f[4] = {v.x, v.y, v.z, v.w};
+        if (keys_ready) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) u[e] = f[e];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) u[e] = i0 + e < vis ? order_key(__uint_as_float(f[e])) : 0u;
+          *reinterpret_cast<uint4*>(keys + i0) = make_uint4(u[0], u[1], u[2], u[3]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (u[e] != 0u) atomicAdd(&hist1[u[e] >> 21], 1u);
+        }
+      }
+      if (!list) continue;
+      uint32_t m[4];
+      int tot = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        m[e] = __ballot_sync(0xFFFFFFFFu, u[e] != 0u && u[e] >= bound);
+        tot += __popc(m[e]);
+      }
+      if (tot == 0) continue;
+      int pos = 0;
+      if ((tid & 31) == 0) pos = atomicAdd(&sel.list_cnt, tot);
+      pos = __shfl_sync(0xFFFFFFFFu, pos, 0);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int q = pos + __popc(m[e] & lt);
+        if ((m[e] >> (tid & 31) & 1u) && q < p.list_cap) list16[q] = static_cast<uint16_t>(i0 + e);
+        pos += __popc(m[e]);
+      }
+    }
+  };
+  auto wait_chunk = [&](int c) -> bool {   // block-uniform: false when the copies gave up
+    if (tid == 0 && !timed_out) {
+      volatile int* flag = &timed_out;
+      mbar_wait(&bars[c], 0, p.budget_ns, flag, p.err);
+    }
+    return !__syncthreads_or(timed_out);
+  };
+  bool ok = true;
+  for (int c = 0; c < nchunks && ok; ++c) {
+    ok = wait_chunk(c);
+    if (!ok) break;
+    if (tr && tid == 0 && c == 0) tr[1] = globaltimer_ns();
+    const int lo = c * kRowChunk, hi = min(lo + kRowChunk, n4);
+    if (c == 0 && use_list) {
+      // the first chunk alone sets the bound (1.5 × its expected share of the k
+      // best), then its keys are listed against it
+      convert(lo, hi, false, false);
+      if (tr && tid == 0) tr[2] = globaltimer_ns();
+      __syncthreads();
+      if (warp == 0) {
+        const int target = row_filter_target(hi, vis, kt);
+        if (target > 0) row_filter_raise_fine(sel, hist1, target);
+      }
+      __syncthreads();
+      if (tr && tid == 0) tr[5] = globaltimer_ns();
+      convert(lo, hi, true, true);
+    } else {
+      if (c == 2 && use_list && warp == 0) {
+        // raised once more on the first two chunks' counts (complete: every warp
+        // passed the barrier of this chunk's wait)
+        const int target = row_filter_target(lo, vis, kt);
+        if (target > 0) row_filter_raise_fine(sel, hist1, target);
+      }
+      convert(lo, hi, use_list, false);
+    }
+    if (tr && tid == 0 && c == 0) tr[6] = globaltimer_ns();
+  }
+  if (!ok) {
+    // give up on this row: let every copy land (bounded) before the CTA exits
+    if (tid == 0) {
+      int dummy = 0;
+      for (int d = 0; d < nchunks; ++d) mbar_wait(&bars[d], 0, p.budget_ns, &dummy, p.err);
+    }
+    __syncthreads();
+    for (int t = tid; t < p.k; t += nthr) out[t] = -1;
+    return;
+  }
+  __syncthreads();
+  if (tid < 64) {   // level-1 coarse sums
+    const uint4* h = reinterpret_cast<const uint4*>(hist1 + 32 * tid);
+    uint32_t sum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint4 v = h[q];
+      sum += v.x + v.y + v.z + v.w;
+    }
+    sel.coarse[0][tid] = sum;
+  }
+  __syncthreads();
+  if (tr && tid == 0) tr[3] = globaltimer_ns();
+  cta_select_row(sel, keys, vis, 0, kt, hist1, true, use_list ? list16 : nullptr, p.list_cap, cand16, p.cand_cap,
+                 out, nullptr, tr, nullptr);
+  for (int t = kt + tid; t < p.k; t += nthr) out[t] = -1;
+  if (tr && tid == 0) tr[4] = globaltimer_ns();
+}
+
 int pow2_floor_i(int x) {
   int r = 1;
   while (r * 2 <= x) r *= 2;
@@ -126,6 +321,32 @@ extern "C" int idx_topk(const float* scores, const int32_t* lengths, int B, int 
   if (max_len < n || max_len > IDX_MAX_LEN || static_cast<int64_t>(max_len) > ld) return IDX_ERR_SHAPE;
   const int64_t rows = static_cast<int64_t>(B) * n;
   const int sms = num_sms();
+  // one CTA per row when the row fits a CTA and enough rows cover the GPU:
+  // bulk copies need 16-byte aligned rows
+  const bool aligned = (reinterpret_cast<uintptr_t>(scores) & 15u) == 0 && (ld & 3) == 0;
+  if (aligned && max_len <= kRowChunk * kRowMaxChunks && (rows >= 64 || rows * 2 >= sms) && rows <= 0x7FFFFFFF) {
+    const int chunk_cap = (max_len + 3) & ~3;
+    const int list_cap = chunk_cap >= 4 * k ? (min(6144, chunk_cap / 2) & ~3) : 0;
+    const int cand_cap = min(2048, chunk_cap);
+    const RowLayout L = row_layout(chunk_cap, list_cap, cand_cap);
+    const int smem = L.total + 128;
+    if (smem > max_dynamic_smem()) return IDX_ERR_SHAPE;
+    static int configured_row = -1;
+    if (configured_row < smem) {
+      if (cudaFuncSetAttribute(topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return check_launch();
+      configured_row = smem;
+    }
+    const DebugState dbg = debug_state();
+    RowParams rp{scores, lengths, indices, ld, B, n, max_len, causal, k, chunk_cap, list_cap, cand_cap,
+                 dbg.budget_ns, device_error_word(), (dbg.flags & 2u) ? trace_buffer() : nullptr};
+    if (!rp.err) return check_launch();
+    // long rows: 16 warps per CTA hide shared-memory latency; short rows: more CTAs per SM
+    const int threads = chunk_cap > 2 * kRowChunk ? kRowThreads : kTopkThreads;
+    topk_row_kernel<<<static_cast<unsigned>(rows), threads, static_cast<size_t>(smem),
+                      reinterpret_cast<cudaStream_t>(stream)>>>(rp);
+    return check_launch();
+  }
   int G = rows < sms ? pow2_floor_i(static_cast<int>(sms / rows)) : 1;
   if (G > 8) G = 8;
   while (G > 1 && (max_len + G - 1) / G < 512) G /= 2;

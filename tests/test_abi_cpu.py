@@ -17,7 +17,8 @@ def _declared():
 
 def test_header_declares_the_boundary():
     names = _declared()
-    for n in ["idx_quant", "idx_quant_append", "idx_score", "idx_topk", "idx_score_topk", "idx_workspace_size",
+    for n in ["idx_quant", "idx_quant_append", "idx_score", "idx_score_visible", "idx_topk", "idx_score_topk",
+              "idx_workspace_size",
               "idx_status", "idx_error_string"]:
         assert n in names
 

@@ -80,3 +80,46 @@ def test_logits_exact_single_head_probe():
         ratio = (err / np.maximum(mag, 1e-30)).max()
         print(f"head {h}: max |err| / sum|q*k| = {ratio:.3e} (2^{np.log2(max(ratio, 1e-300)):.2f})")
         assert np.all(err <= 2.0 ** -20 * mag + 1e-30), err.max()
+
+
+VISIBLE = [
+    # name, B, n, positions, T_cap, causal, fmt — decode batches, ragged and zero
+    # lengths, causal and chunked prefill, more row blocks than SMs
+    ("decode-batch", 150, 1, None, 2048, False, 1),
+    ("decode-ragged", 5, 1, [0, 126, 128, 999, 4095], 4096, False, 0),
+    ("prefill-causal", 1, 300, [0], 512, True, 0),
+    ("prefill-chunked", 2, 261, [200, 517], 1024, True, 1),
+    ("many-blocks", 3, 200, [0, 100, 600], 1024, True, 0),
+]
+
+
+@pytest.mark.parametrize("name,B,n,positions,T_cap,causal,fmt", VISIBLE)
+def test_score_visible_matches_oracle(name, B, n, positions, T_cap, causal, fmt):
+    """idx_score_visible (flat partition, one persistent CTA per SM): the oracle's
+    scores on every visible key, −inf up to the end of each row's last key tile."""
+    from sparse_attention_token_idx_b200 import binding as X
+    kw = dict(lengths_draw=(1, T_cap - 1)) if positions is None else {}
+    case = synth.make_case(name, 250 + len(name), B, n, positions, T_cap=T_cap, causal=causal, fmt=fmt, **kw)
+    kc, ks, lengths = gpu_state(case)
+    qc, w = gpu_queries(case)
+    max_len = int(case.lengths.max())
+    ld = max_len + 5
+    out = torch.full((B, n, ld), 12345.0, dtype=torch.float32, device="cuda")
+    X.score_visible(qc, w, kc, ks, lengths, causal, max_len, ld=ld, out=out)
+    assert X.status() == (0, 0)
+    got = out.cpu().numpy()
+    okc, oks = oracle_state(case)
+    oqc, ow = oracle_queries(case)
+    S, E = O.index_scores(oqc, ow, okc, oks, case.lengths, causal, ncols=ld)
+    for b in range(B):
+        blocks = {}
+        for i in range(n):
+            vis = O.visible_count(int(case.lengths[b]), n, i, causal)
+            blk = i // 4 if n > 2 else i
+            blocks[blk] = max(blocks.get(blk, 0), vis)
+        for i in range(n):
+            vis = O.visible_count(int(case.lengths[b]), n, i, causal)
+            end = min(ld, -(-blocks[i // 4 if n > 2 else i] // 128) * 128)   # the row block's last key tile
+            check_scores(got[b, i:i + 1, :vis][None], S[b, i:i + 1, :vis][None], E[b, i:i + 1, :vis][None])
+            assert np.all(np.isneginf(got[b, i, vis:end])), "−inf up to the end of the last key tile"
+            assert np.all(got[b, i, end:] == 12345.0), "columns past the last key tile untouched"

@@ -36,6 +36,40 @@ def test_topk_exact(B, n, lengths, causal, k, ties):
             check_topk_exact_row(got[b, i], sc[b, i], vis, k)
 
 
+# Many rows: one CTA per row, rows fetched by bulk copies, the candidate list
+# kept while the keys are counted (used when the k best are a small share).
+ROWS = [
+    # name, rows, longest row, ld, k, score order
+    ("gauss", 128, 16384, 16384, 2048, "random"),
+    ("ties", 96, 12000, 12000, 2048, "ties"),          # bin-b1 candidates overflow their list
+    ("best-first", 64, 16384, 16384, 2048, "desc"),    # the early bound overshoots: slice fallback
+    ("best-last", 64, 16384, 16384, 2048, "asc"),      # the list overflows: slice fallback
+    ("large-k", 64, 16384, 16384, 4096, "random"),     # positions written without staging
+    ("ragged", 80, 16381, 16384, 512, "random"),       # lengths not multiples of 4 (ld is)
+    ("unaligned-ld", 70, 3001, 3001, 700, "random"),   # ld % 4 != 0: cluster kernel
+]
+
+
+@pytest.mark.parametrize("name,rows,L,ld,k,order", ROWS)
+def test_topk_many_rows(name, rows, L, ld, k, order):
+    from sparse_attention_token_idx_b200 import binding as X
+    rng = np.random.default_rng(rows * 7 + L + k)
+    sc = rng.standard_normal((rows, 1, ld)).astype(np.float32)
+    if order == "ties":
+        sc = np.round(sc * 4) / 4
+    elif order == "desc":
+        sc = sc - np.float32(0.01) * np.arange(ld, dtype=np.float32)
+    elif order == "asc":
+        sc = sc + np.float32(0.01) * np.arange(ld, dtype=np.float32)
+    lengths = rng.integers(max(1, L - 700), L + 1, rows).astype(np.int32)
+    lengths[0] = L
+    lengths[1] = min(L, k)                       # every visible key selected
+    got = X.topk(dev(sc), dev(lengths), False, k, L).cpu().numpy()
+    assert X.status() == (0, 0)
+    for r in range(rows):
+        check_topk_exact_row(got[r, 0], sc[r, 0], int(lengths[r]), k)
+
+
 def test_topk_negative_zero_and_infinities():
     from sparse_attention_token_idx_b200 import binding as X
     s = np.array([[[0.0, -0.0, 1.0, -np.inf, np.inf, -1.0, 0.0, -0.0]]], np.float32)
@@ -51,6 +85,9 @@ FUSED = [
     ("decode-small-k", 4, 1, [511, 2000, 777, 3333], 4096, False, 0, 17),
     ("prefill", 1, 300, [0], 512, True, 0, 64),
     ("chunked", 2, 130, [900, 2500], 4096, True, 1, 512),
+    # 64 decode rows: with a workspace the scorer splits rows over plain CTAs
+    # and the top-k takes one row per CTA
+    ("decode-many", 64, 1, list(range(1000, 2024, 16)), 2048, False, 1, 256),
 ]
 
 
