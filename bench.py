@@ -39,7 +39,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FP8_PER_BF16 = 2.0            # nominal dense fp8 : bf16 tensor ratio on B200
 KEY_BYTES = 128 + 4           # one cached key: 128 e4m3 codes + fp32 scale
 ROW_BYTES_IN = 64 * 128 + 64 * 4   # one query row: 64 heads of e4m3 codes + 64 fp32 weights
-PROFILE_SCORE = os.path.join(ROOT, "profiles", "score_decode_b128_t16384.md")
+PROFILE_SCORE = os.path.join(ROOT, "profiles", "score_topk_decode_b128_t16384.md")
 KERNEL_SOURCES = ["score.cu", "select.cuh", "ptx.cuh"]
 
 

@@ -360,22 +360,25 @@ __global__ void __launch_bounds__(FCfg<NT, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W
                      pack2(fmaxf(__uint_as_float(r1[2 * i]), 0.f), fmaxf(__uint_as_float(r1[2 * i + 1]), 0.f)),
                      wp[16 + i]);
             } else {
+              // both halves in flight before one wait; weights from shared memory
+              uint32_t r[2][32];
+              tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64), r[0]);
+              tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64 + 32), r[1]);
+              tmem_wait();
+              tmem_regs_ready(r[0]);
+              tmem_regs_ready(r[1]);
 #pragma unroll
               for (int c = 0; c < 2; ++c) {
-                uint32_t r0[32];
-                tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64 + c * 32), r0);
-                tmem_wait();
-                tmem_regs_ready(r0);
                 const float4* wv = reinterpret_cast<const float4*>(wrow + j * 64 + c * 32);
 #pragma unroll
                 for (int i4 = 0; i4 < 8; ++i4) {
                   const float4 w4 = wv[i4];
                   fma2(acc[(2 * i4) & 3],
-                       pack2(fmaxf(__uint_as_float(r0[4 * i4]), 0.f), fmaxf(__uint_as_float(r0[4 * i4 + 1]), 0.f)),
+                       pack2(fmaxf(__uint_as_float(r[c][4 * i4]), 0.f), fmaxf(__uint_as_float(r[c][4 * i4 + 1]), 0.f)),
                        pack2(w4.x, w4.y));
                   fma2(acc[(2 * i4 + 1) & 3],
-                       pack2(fmaxf(__uint_as_float(r0[4 * i4 + 2]), 0.f),
-                             fmaxf(__uint_as_float(r0[4 * i4 + 3]), 0.f)),
+                       pack2(fmaxf(__uint_as_float(r[c][4 * i4 + 2]), 0.f),
+                             fmaxf(__uint_as_float(r[c][4 * i4 + 3]), 0.f)),
                        pack2(w4.z, w4.w));
                 }
               }
