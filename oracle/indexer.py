@@ -28,6 +28,10 @@ What it computes, step by step, with the passage each step follows:
 * ``topk``             — ``Indexer.forward`` excerpt (top min(index_topk, ·)
   positions per row) and the NKI "DeepSeek-V3.2 Sparse Indexer Kernel API
   Reference" page, Notes and return types (int32, an unordered set).
+* ``e8m0_encode`` / ``e8m0_decode`` — the power-of-two key scale stored as one
+  byte, the "e8m0" of the ``fp8_index`` docstring ("Index scores" page).
+* ``MASK_BOUND_BF16``, ``scores_bf16`` — the NKI page's Notes: masked slots
+  hold a finite bound instead of −inf for consumers that read bfloat16.
 
 Readings taken where the pages are silent (each one also listed in the design doc):
 
@@ -45,6 +49,12 @@ Readings taken where the pages are silent (each one also listed in the design doc):
   is visible to it iff s < lengths[b] and, when causal, s ≤ that position.
 * The row keeps k_t = min(k, number of visible keys) positions; the oracle
   orders by score descending, then position ascending, and pads with −1.
+* e8m0 is the OCP MX scale format: an unsigned biased exponent, value
+  2^(byte − 127), no sign or mantissa (0xFF not used).
+* The finite mask bound, whose value the NKI page does not give, is the most
+  negative finite bfloat16, −(2 − 2^−7) · 2^127 — exact in bf16 and fp32, so
+  a bf16 consumer reads it unchanged.
+* A bf16 score is the round-to-nearest-even of the fp32 score.
 
 Precision: the FP8 dot products are computed exactly in float64 (every product
 of two e4m3 values is a multiple of 2^-18 below 2^17.7, so a 128-term sum needs
@@ -269,6 +279,38 @@ def index_scores(q_codes, w, k_cache, k_scale_cache, lengths, causal, ncols=None
             if with_bound:
                 E[b, i, :v] = np.abs(ks[:v]) * np.sum(np.abs(wi * logits), axis=0)
     return S, E
+
+
+# --------------------------------------------------------------------------- variants
+# e8m0 (OCP MX scale format): one byte, value 2^(byte − 127).
+def e8m0_encode(scale: np.ndarray) -> np.ndarray:
+    """Byte of a positive power-of-two scale in [2^-127, 2^127]; raises otherwise."""
+    s = np.asarray(scale, np.float64)
+    m, e = np.frexp(s)                 # s = m · 2^e with m in [0.5, 1)
+    if np.any(s <= 0) or np.any(m != 0.5):
+        raise AssertionError("e8m0 holds positive powers of two only")
+    k = e - 1                          # s = 2^k
+    if np.any(k < -127) or np.any(k > 127):
+        raise AssertionError("exponent out of the e8m0 range")
+    return (k + 127).astype(np.uint8)
+
+
+def e8m0_decode(byte: np.ndarray) -> np.ndarray:
+    return np.ldexp(1.0, np.asarray(byte, np.int64) - 127)
+
+
+# The finite mask bound: the most negative finite bfloat16.
+MASK_BOUND_BF16 = -(2.0 - 2.0 ** -7) * 2.0 ** 127
+
+
+def masked(S: np.ndarray, bound: float) -> np.ndarray:
+    """S with its masked (−inf) entries replaced by a finite bound."""
+    return np.where(np.isneginf(S), bound, S)
+
+
+def scores_bf16(S_f32: np.ndarray) -> np.ndarray:
+    """bf16 output of fp32 scores: round to nearest even (values as float64)."""
+    return bf16_round(np.asarray(S_f32, np.float32).astype(np.float64))
 
 
 # --------------------------------------------------------------------------- top-k

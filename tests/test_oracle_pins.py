@@ -462,3 +462,52 @@ def test_append_writes_exactly_the_requested_slots():
         assert np.all(kc[b, mask] == 0xAB) and np.all(ks[b, mask] == -7.0)
     with pytest.raises(ValueError):
         O.quant_append(case.k_new, [0, 0, 29], kc, ks, 1)
+
+
+# ---------------------------------------------------------------- variants
+def test_e8m0_byte_is_the_ieee_exponent_field():
+    """The e8m0 byte of 2^k is the biased exponent field of the fp32 value 2^k
+    (IEEE 754 binary32: bits 30…23, bias 127), for every normal power of two."""
+    ks = np.arange(-126, 128)
+    vals = np.ldexp(1.0, ks)
+    field = (vals.astype(np.float32).view(np.uint32) >> 23) & 0xFF
+    assert np.array_equal(O.e8m0_encode(vals), field.astype(np.uint8))
+    assert np.array_equal(O.e8m0_decode(field), vals)
+    assert O.e8m0_encode(np.array([1.0]))[0] == 127
+
+
+def test_e8m0_round_trips_every_ue8m0_scale_and_rejects_others():
+    rng = np.random.default_rng(5)
+    amax = np.abs(rng.standard_normal(5000)).astype(np.float32) * np.float32(100)
+    amax[:3] = [0.0, 448.0, 3e-5]
+    s = O.scale_from_amax(amax, 1)
+    assert np.array_equal(O.e8m0_decode(O.e8m0_encode(s)), s.astype(np.float64))
+    for bad in (3.0, 0.75, -2.0, 0.0):
+        with pytest.raises(AssertionError):
+            O.e8m0_encode(np.array([bad]))
+
+
+def test_mask_bound_is_the_most_negative_finite_bf16():
+    import torch
+    assert O.MASK_BOUND_BF16 == float(torch.finfo(torch.bfloat16).min)
+    assert O.bf16_round(np.array([O.MASK_BOUND_BF16]))[0] == O.MASK_BOUND_BF16
+    assert float(np.float32(O.MASK_BOUND_BF16)) == O.MASK_BOUND_BF16
+    S = np.array([[1.5, -np.inf, -3.0, -np.inf]])
+    assert np.array_equal(O.masked(S, O.MASK_BOUND_BF16), [[1.5, O.MASK_BOUND_BF16, -3.0, O.MASK_BOUND_BF16]])
+
+
+def test_bf16_scores_match_torch_rounding():
+    """Round-to-nearest-even fp32 → bf16, against torch's conversion (ties,
+    values next to the rounding boundary, subnormals, large magnitudes)."""
+    import torch
+    rng = np.random.default_rng(6)
+    x = (rng.standard_normal(20000) * np.exp(rng.uniform(-40, 40, 20000))).astype(np.float32)
+    u = rng.integers(0, 2 ** 32, 20000, dtype=np.uint64).astype(np.uint32)
+    u = (u & np.uint32(0xFFFF0000)) | np.uint32(0x8000)          # exact ties
+    ties = u.view(np.float32)
+    ties = ties[np.isfinite(ties)]
+    x = np.concatenate([x, ties, np.float32([1e-40, -3e-39, 3.3e38, -3.39e38])])
+    want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    got = O.scores_bf16(x)
+    fin = np.isfinite(want)
+    assert np.array_equal(got[fin], want[fin])
