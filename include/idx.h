@@ -58,6 +58,20 @@ typedef struct CUstream_st* idx_stream_t;
 
 enum idx_fmt { IDX_FMT_FP32 = 0, IDX_FMT_UE8M0 = 1 };
 
+/* Key-scale storage read by the *_ex score calls: fp32 values, or one e8m0
+ * byte per key (OCP MX scale format: value 2^(byte − 127)), as written by
+ * idx_quant_append_e8 — 129 instead of 132 cache bytes per key. */
+enum idx_scale_storage { IDX_SCALE_F32 = 0, IDX_SCALE_E8M0 = 1 };
+
+/* Score element type written by idx_score_ex. */
+enum idx_score_dtype { IDX_SCORE_F32 = 0, IDX_SCORE_BF16 = 1 };
+
+/* The most negative finite bfloat16, −(2 − 2^−7)·2^127: a finite mask value a
+ * bf16 consumer reads unchanged ("DeepSeek-V3.2 Sparse Indexer Kernel API
+ * Reference" page, Notes: masked slots are clamped to a finite bound because a
+ * bf16 max-select turns −inf into NaN).  Exact in fp32. */
+#define IDX_MASK_BOUND_BF16 (-3.38953138925153547590470800371487866880e+38f)
+
 enum idx_status_code {
   IDX_OK = 0,
   IDX_ERR_NULL = -1,        /* a required pointer is NULL */
@@ -115,6 +129,16 @@ IDX_API int idx_quant_append(const uint16_t* k_bf16, const int32_t* positions, i
                      float* k_scale_cache, int T_cap, int fmt, idx_stream_t stream);
 
 /*
+ * idx_quant_append_e8 — idx_quant_append with fmt = IDX_FMT_UE8M0 and each key's
+ * power-of-two scale stored as its e8m0 byte (2^(byte − 127); the byte is the
+ * fp32 exponent field of the scale) in k_scale_e8 [B, T_cap] uint8 — the "e8m0"
+ * of the fp8_index docstring ("Index scores" page).  Read by the *_ex score
+ * calls with IDX_SCALE_E8M0.  Arguments, alignment and errors as idx_quant_append.
+ */
+IDX_API int idx_quant_append_e8(const uint16_t* k_bf16, const int32_t* positions, int B, int n, uint8_t* k_cache,
+                                uint8_t* k_scale_e8, int T_cap, idx_stream_t stream);
+
+/*
  * idx_quant_queries_append — idx_quant_queries and idx_quant_append of one
  * indexer call in a single launch (the two are independent row sets of the
  * same rotation + quantisation).  Arguments as in the two calls; either part
@@ -140,6 +164,25 @@ IDX_API int idx_quant_queries_append(const uint16_t* q_bf16, const float* w_raw,
 IDX_API int idx_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
               const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, float* scores, int64_t ld,
               idx_stream_t stream);
+
+/*
+ * idx_score_ex — idx_score with the storage and output options of the NKI
+ * indexer page (its Notes on the finite mask bound) and of the fp8_index
+ * docstring (the key scale "e8m0 here"):
+ *   k_scale      [B, T_cap] key scales: float32 (scale_fmt = IDX_SCALE_F32) or
+ *                uint8 e8m0 bytes (IDX_SCALE_E8M0; T_cap a multiple of 16),
+ *                16-byte aligned.
+ *   scores       [B, n, ld] of score_dtype: IDX_SCORE_F32, or IDX_SCORE_BF16
+ *                (each fp32 score rounded to nearest even).
+ *   mask_value   written to every masked column: −inf as idx_score, or a
+ *                finite bound such as IDX_MASK_BOUND_BF16 (NaN is rejected).
+ * An e8m0 scale is the same power of two as the fp32 ue8m0 scale, so the
+ * scores equal idx_score's on a cache filled with IDX_FMT_UE8M0.
+ * Returns IDX_ERR_FMT for an unknown scale_fmt or score_dtype.
+ */
+IDX_API int idx_score_ex(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const void* k_scale,
+                         int scale_fmt, const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal,
+                         void* scores, int64_t ld, int score_dtype, float mask_value, idx_stream_t stream);
 
 /*
  * idx_score_visible — the scores of idx_score for the visible keys only, as
@@ -179,6 +222,16 @@ IDX_API int idx_topk(const float* scores, const int32_t* lengths, int B, int n, 
 IDX_API int idx_score_topk(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
                    const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, int k,
                    int32_t* indices, void* ws, size_t ws_bytes, idx_stream_t stream);
+
+/*
+ * idx_score_topk_ex — idx_score_topk with the key scales stored as fp32
+ * (scale_fmt = IDX_SCALE_F32) or as e8m0 bytes (IDX_SCALE_E8M0, T_cap a
+ * multiple of 16).  The selected set equals idx_score_topk's on a cache filled
+ * with IDX_FMT_UE8M0.
+ */
+IDX_API int idx_score_topk_ex(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const void* k_scale,
+                              int scale_fmt, const int32_t* lengths, int B, int n, int T_cap, int max_len,
+                              int causal, int k, int32_t* indices, void* ws, size_t ws_bytes, idx_stream_t stream);
 
 /*
  * idx_score_topk_noalloc — idx_score_topk for callers that cannot allocate

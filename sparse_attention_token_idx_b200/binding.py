@@ -23,6 +23,11 @@ DIM = 128
 DEV_ERR_TIMEOUT = 0x1
 DEV_ERR_POSITION = 0x2
 DEV_ERR_LENGTH = 0x4
+SCALE_F32 = 0
+SCALE_E8M0 = 1
+SCORE_F32 = 0
+SCORE_BF16 = 1
+MASK_BOUND_BF16 = -3.3895313892515355e38    # most negative finite bfloat16
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -35,11 +40,14 @@ SIGNATURES = {
     "idx_quant_queries": (_I, [_P, _P, _I64, _P, _P, _I, _P]),
     "idx_quant_append": (_I, [_P, _P, _I, _I, _P, _P, _I, _I, _P]),
     "idx_quant_queries_append": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _I, _P, _P, _I, _I, _P]),
+    "idx_quant_append_e8": (_I, [_P, _P, _I, _I, _P, _P, _I, _P]),
     "idx_score": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P]),
     "idx_score_visible": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P]),
+    "idx_score_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _P, _I64, _I, ctypes.c_float, _P]),
     "idx_topk": (_I, [_P, _P, _I, _I, _I64, _I, _I, _I, _P, _P, _SZ, _P]),
     "idx_score_topk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "idx_score_topk_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
+    "idx_score_topk_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "idx_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "idx_status": (_I, [_P]),
     "idx_device_error_bits": (ctypes.c_uint, []),
@@ -172,6 +180,53 @@ def score_visible(q_fp8, w, k_cache, k_scale_cache, lengths, causal: bool, max_l
                                     _ptr(k_scale_cache, torch.float32, "k_scale"),
                                     _ptr(lengths, torch.int32, "lengths"), B, n, T_cap, max_len, int(causal),
                                     _ptr(out, torch.float32, "scores"), ld, _stream(stream)), "idx_score_visible")
+    return out
+
+
+def quant_append_e8(k_new, positions, k_cache, k_scale_e8, stream=None):
+    """Rotate, quantise (ue8m0) and append keys; scales stored as e8m0 bytes."""
+    B, n = k_new.shape[0], k_new.shape[1]
+    _check(load().idx_quant_append_e8(_ptr(k_new, _BF16, "k_new"), _ptr(positions, torch.int32, "positions"),
+                                      B, n, _ptr(k_cache, torch.uint8, "k_cache"),
+                                      _ptr(k_scale_e8, torch.uint8, "k_scale_e8"), k_cache.shape[1],
+                                      _stream(stream)), "idx_quant_append_e8")
+
+
+def _scale_arg(k_scale):
+    if k_scale.dtype == torch.uint8:
+        return _ptr(k_scale, torch.uint8, "k_scale"), SCALE_E8M0
+    return _ptr(k_scale, torch.float32, "k_scale"), SCALE_F32
+
+
+def score_ex(q_fp8, w, k_cache, k_scale, lengths, causal: bool, max_len: int, ld: int | None = None,
+             dtype=torch.float32, mask_value: float = float("-inf"), out=None, stream=None):
+    """Scores [B, n, ld] in fp32 or bf16 with a chosen mask value; key scales fp32
+    or e8m0 bytes (uint8)."""
+    B, n = q_fp8.shape[0], q_fp8.shape[1]
+    T_cap = k_cache.shape[1]
+    ld = ld if ld is not None else max_len
+    out = out if out is not None else torch.empty((B, n, ld), dtype=dtype, device=q_fp8.device)
+    sdt = SCORE_BF16 if out.dtype == torch.bfloat16 else SCORE_F32
+    ks, sfmt = _scale_arg(k_scale)
+    _check(load().idx_score_ex(_ptr(q_fp8, torch.uint8, "q_fp8"), _ptr(w, torch.float32, "w"),
+                               _ptr(k_cache, torch.uint8, "k_cache"), ks, sfmt, _ptr(lengths, torch.int32, "lengths"),
+                               B, n, T_cap, max_len, int(causal), _ptr(out, out.dtype, "scores"), ld, sdt,
+                               float(mask_value), _stream(stream)), "idx_score_ex")
+    return out
+
+
+def score_topk_ex(q_fp8, w, k_cache, k_scale, lengths, causal: bool, k: int, max_len: int, out=None,
+                  ws: torch.Tensor | None = None, stream=None):
+    """score_topk with key scales fp32 or e8m0 bytes (uint8)."""
+    B, n = q_fp8.shape[0], q_fp8.shape[1]
+    out = out if out is not None else torch.empty((B, n, k), dtype=torch.int32, device=q_fp8.device)
+    ks, sfmt = _scale_arg(k_scale)
+    wsp, wsn = (None, 0) if ws is None else (_ptr(ws, None, "ws"), ws.numel() * ws.element_size())
+    _check(load().idx_score_topk_ex(_ptr(q_fp8, torch.uint8, "q_fp8"), _ptr(w, torch.float32, "w"),
+                                    _ptr(k_cache, torch.uint8, "k_cache"), ks, sfmt,
+                                    _ptr(lengths, torch.int32, "lengths"), B, n, k_cache.shape[1], max_len,
+                                    int(causal), k, _ptr(out, torch.int32, "indices"), wsp, wsn, _stream(stream)),
+           "idx_score_topk_ex")
     return out
 
 

@@ -137,6 +137,26 @@ bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner) {
+  resolve_encode();
+  if (!g_encode) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || (inner & 15)) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner};
+  const cuuint32_t box[2] = {box_inner, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_scales(CUtensorMap* map, const void* base, int scale_fmt, uint64_t T_cap, uint64_t B,
+                      uint32_t box_inner) {
+  return scale_fmt == kScaleE8M0 ? make_tmap_u8_2d(map, base, T_cap, B, box_inner)
+                                 : make_tmap_f32_2d(map, base, T_cap, B, box_inner);
+}
+
 DebugState debug_state() {
   DebugState s;
   s.flags = g_debug_flags.load();

@@ -24,15 +24,31 @@ unsigned int* device_error_word();  // device address of the error word on the c
 // multiple of 16), box {box_inner, 1}, no swizzle.
 bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner);
 
+// Tensor map for a [outer, inner] uint8 array (row pitch inner bytes, a
+// multiple of 16), box {box_inner, 1}, no swizzle.
+bool make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner);
+
+// Key-scale storage of a score call: fp32 values, or e8m0 bytes (2^(byte − 127)).
+enum { kScaleF32 = 0, kScaleE8M0 = 1 };
+
+// Options of a score call beyond the method's definition.
+struct ScoreVariant {
+  int scale_fmt;      // kScaleF32 or kScaleE8M0
+  int out_bf16;       // unfused scores in bf16 (round to nearest even) instead of fp32
+  float mask_value;   // unfused scores: value of masked columns (−inf, or a finite bound)
+};
+bool make_tmap_scales(CUtensorMap* map, const void* base, int scale_fmt, uint64_t T_cap, uint64_t B,
+                      uint32_t box_inner);
+
 unsigned long long* trace_buffer();  // device address of the phase-trace buffer
 
 // Flat-partition scorer (flat_score.cu): scores of every visible (row, key) of
 // the call into scores [B, n, ld], one persistent CTA per SM; columns past a
 // row's last key tile are left unwritten.  IDX_ERR_UNSUPPORTED when the call
 // has more row blocks than the kernel's shared-memory index holds.
-int launch_flat_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
-                      const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, float* scores,
-                      int64_t ld, cudaStream_t stream);
+int launch_flat_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const void* k_scale_cache,
+                      int scale_fmt, const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal,
+                      float* scores, int64_t ld, cudaStream_t stream);
 
 struct DebugState {
   unsigned int flags;

@@ -50,6 +50,7 @@ struct FlatParams {
   unsigned long long budget_ns;
   unsigned int* err;
   unsigned long long* trace;   // per-CTA phase stamps (16 slots), or null
+  int scale_u8;                // key scales stored as e8m0 bytes (else fp32)
 };
 
 template <int NT, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT, bool W_REGS>
@@ -251,7 +252,7 @@ __global__ void __launch_bounds__(FCfg<NT, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W
         const int c = k % kFScaleSlots;
         if (!mbar_wait(&empty[s], ((k / STAGES) & 1) ^ 1, budget, abort_flag, p.err)) break;
         if (!mbar_wait(&sc_empty[c], ((k / kFScaleSlots) & 1) ^ 1, budget, abort_flag, p.err)) break;
-        mbar_arrive_expect_tx(&full[s], kFTileBytes + kFKeys * 4);
+        mbar_arrive_expect_tx(&full[s], kFTileBytes + kFKeys * (p.scale_u8 ? 1 : 4));
         tma_load_3d(k_s + s * kFTileBytes, &tmap_k, &full[s], 0, wk.tile * kFKeys, blk.b);
         tma_load_2d(scale_s + c * kFKeys, &tmap_s, &full[s], wk.tile * kFKeys, blk.b);
         tma_issued = k + 1;
@@ -334,7 +335,10 @@ __global__ void __launch_bounds__(FCfg<NT, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W
           if (!__shfl_sync(0xFFFFFFFFu, ok, 0)) break;
           if (tr && k == 0 && ew == 0 && lane == 0) tr[2] = globaltimer_ns();
           tc_fence_after();
-          const float ks = scale_s[c * kFKeys + kl];   // landed with the keys (same barrier)
+          // landed with the keys (same barrier); an e8m0 byte is the exponent field of its value
+          const float ks = p.scale_u8 ? __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint8_t*>(
+                                            scale_s + c * kFKeys)[kl]) << 23)
+                                      : scale_s[c * kFKeys + kl];
           const int key = wk.tile * kFKeys + kl;
           const float* wrow = w_s + (qseq & 1) * N;
 #pragma unroll
@@ -431,9 +435,9 @@ __global__ void __launch_bounds__(FCfg<NT, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W
 }
 
 template <int NT, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT, bool W_REGS>
-int launch_flat_t(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
-                  const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, float* scores,
-                  int64_t ld, cudaStream_t stream) {
+int launch_flat_t(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const void* k_scale_cache,
+                  int scale_fmt, const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal,
+                  float* scores, int64_t ld, cudaStream_t stream) {
   using C = FCfg<NT, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>;
   const int ntb = (n + NT - 1) / NT;
   const int64_t items = static_cast<int64_t>(B) * ntb;
@@ -446,7 +450,7 @@ int launch_flat_t(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, 
     return IDX_ERR_ALIGN;
   if (!make_tmap_u8_3d(&tq, q_fp8, IDX_DIM, static_cast<uint64_t>(n) * IDX_HEADS, static_cast<uint64_t>(B), C::N))
     return IDX_ERR_ALIGN;
-  if (!make_tmap_f32_2d(&ts, k_scale_cache, static_cast<uint64_t>(T_cap), static_cast<uint64_t>(B), kFKeys))
+  if (!make_tmap_scales(&ts, k_scale_cache, scale_fmt, static_cast<uint64_t>(T_cap), static_cast<uint64_t>(B), kFKeys))
     return IDX_ERR_ALIGN;
   auto kern = flat_score_kernel<NT, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>;
   static int configured_smem = -1;   // per instantiation
@@ -471,6 +475,7 @@ int launch_flat_t(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, 
   p.budget_ns = dbg.budget_ns;
   p.err = device_error_word();
   p.trace = (dbg.flags & 2u) ? trace_buffer() : nullptr;
+  p.scale_u8 = scale_fmt == kScaleE8M0 ? 1 : 0;
   if (!p.err) return check_launch();
   kern<<<static_cast<unsigned>(num_sms()), C::kThreads, static_cast<size_t>(smem), stream>>>(tk, tq, ts, p);
   return check_launch();
@@ -480,14 +485,14 @@ int launch_flat_t(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, 
 
 // Scores of every visible (row, key) of the call into `scores` [B, n, ld]
 // (columns past each row block's last key tile left as they were).
-int launch_flat_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const float* k_scale_cache,
-                      const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal, float* scores,
-                      int64_t ld, cudaStream_t stream) {
+int launch_flat_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, const void* k_scale_cache,
+                      int scale_fmt, const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal,
+                      float* scores, int64_t ld, cudaStream_t stream) {
   if (n <= 2)
-    return launch_flat_t<1, 6, 4, 8, 2, true>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
-                                        scores, ld, stream);
-  return launch_flat_t<4, 4, 2, 16, 1, false>(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal,
-                                       scores, ld, stream);
+    return launch_flat_t<1, 6, 4, 8, 2, true>(q_fp8, w, k_cache, k_scale_cache, scale_fmt, lengths, B, n, T_cap,
+                                              max_len, causal, scores, ld, stream);
+  return launch_flat_t<4, 4, 2, 16, 1, false>(q_fp8, w, k_cache, k_scale_cache, scale_fmt, lengths, B, n, T_cap,
+                                              max_len, causal, scores, ld, stream);
 }
 
 }  // namespace idx

@@ -149,6 +149,7 @@ struct QuantArgs {
   const int32_t* positions;
   uint8_t* k_cache;
   float* k_scale_cache;
+  uint8_t* k_scale_e8;    // instead of k_scale_cache: the scale's e8m0 byte (ue8m0 only)
   int64_t k_rows;
   int n, T_cap;
   int fmt;
@@ -196,7 +197,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) quant_kernel(const QuantA
       d[1] = out.codes[1];
       if (q == 0) {
         if (is_key) {
-          a.k_scale_cache[slot] = out.scale;
+          // a ue8m0 scale is a normal power of two: its byte is the fp32 exponent field
+          if (a.k_scale_e8) a.k_scale_e8[slot] = static_cast<uint8_t>(__float_as_uint(out.scale) >> 23);
+          else a.k_scale_cache[slot] = out.scale;
         } else if (a.w_raw) {
           a.w_out[r] = __fmul_rn(__fmul_rn(__fmul_rn(a.w_raw[r], 0.125f), out.scale),
                                  __uint_as_float(kInvSqrtDfBits));
@@ -301,6 +304,26 @@ extern "C" int idx_quant_queries_append(const uint16_t* q_bf16, const float* w_r
     a.err = device_error_word();
     if (!a.err) return check_launch();
   }
+  return launch_quant(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int idx_quant_append_e8(const uint16_t* k_bf16, const int32_t* positions, int B, int n,
+                                   uint8_t* k_cache, uint8_t* k_scale_e8, int T_cap, idx_stream_t stream) {
+  if (B < 0 || n < 0 || T_cap <= 0) return IDX_ERR_SHAPE;
+  if (B == 0 || n == 0) return IDX_OK;
+  if (n > T_cap) return IDX_ERR_SHAPE;
+  if (!k_bf16 || !positions || !k_cache || !k_scale_e8) return IDX_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(k_bf16) | reinterpret_cast<uintptr_t>(k_cache)) & 15) return IDX_ERR_ALIGN;
+  QuantArgs a = empty_args(IDX_FMT_UE8M0);
+  a.k = k_bf16;
+  a.positions = positions;
+  a.k_cache = k_cache;
+  a.k_scale_e8 = k_scale_e8;
+  a.k_rows = static_cast<int64_t>(B) * n;
+  a.n = n;
+  a.T_cap = T_cap;
+  a.err = device_error_word();
+  if (!a.err) return check_launch();
   return launch_quant(a, reinterpret_cast<cudaStream_t>(stream));
 }
 

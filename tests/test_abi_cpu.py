@@ -50,6 +50,14 @@ def test_host_argument_checks_run_before_any_device_work():
     assert lib.idx_score_topk(None, None, None, None, None, 1, 1, 16, 16, 0, 0, None, None, 0, None) == -1
     assert lib.idx_topk(None, None, 1, 1, 16, 16, 0, 0, None, None, 0, None) == -4
     assert lib.idx_quant_append(None, None, -1, 1, None, None, 16, 0, None) == -2
+    # the variant calls: unknown scale storage / score type, an e8m0 pitch that TMA cannot read
+    p16 = 1 << 20                                   # a 16-byte aligned dummy address, never dereferenced
+    assert lib.idx_score_ex(p16, p16, p16, p16, 2, p16, 1, 1, 16, 16, 0, p16, 16, 0, 0.0, None) == -3
+    assert lib.idx_score_ex(p16, p16, p16, p16, 0, p16, 1, 1, 16, 16, 0, p16, 16, 5, 0.0, None) == -3
+    assert lib.idx_score_ex(p16, p16, p16, p16, 1, p16, 1, 1, 20, 16, 0, p16, 16, 0, 0.0, None) == -2
+    assert lib.idx_score_ex(p16, p16, p16, p16, 0, p16, 1, 1, 16, 16, 0, p16, 16, 0, float("nan"), None) == -2
+    assert lib.idx_score_topk_ex(p16, p16, p16, p16, 3, p16, 1, 1, 16, 16, 0, 8, p16, None, 0, None) == -3
+    assert lib.idx_quant_append_e8(None, None, 1, 1, None, None, 16, None) == -1
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
