@@ -165,7 +165,10 @@ def run_ours(args, rank, world, local_rank):
     bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
     dv = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
 
-    ix = Indexer(B, case.T_cap, case.fmt, case.k, device=dev)
+    e8m0 = getattr(args, "scale_storage", "f32") == "e8m0"
+    if e8m0 and (case.fmt != 1 or case.n > 2):
+        raise SystemExit("--scale-storage e8m0 applies to the ue8m0 decode workload (2)")
+    ix = Indexer(B, case.T_cap, case.fmt, case.k, device=dev, scale_storage="e8m0" if e8m0 else "f32")
     P = case.k_prior.shape[1]
     if P:
         if np.all(case.positions == P):
@@ -184,6 +187,8 @@ def run_ours(args, rank, world, local_rank):
     w = torch.empty(w_raw.shape, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     keys, flops, key_rows, score_bytes = workload_numbers(case)
+    if e8m0:   # one scale byte per cached key instead of four
+        score_bytes -= 3 * key_rows
 
     # the kernel the roofline is about, timed on its own stream with events: the
     # tcgen05 scorer writing the workspace when the step uses one (the step's
@@ -199,7 +204,7 @@ def run_ours(args, rank, world, local_rank):
             X.score_visible(q_fp8, w, ix.k_cache, ix.k_scale_cache, lengths, case.causal, max_len, ld=max_len,
                             out=sc_view)
         else:
-            X.score_topk(q_fp8, w, ix.k_cache, ix.k_scale_cache, lengths, case.causal, case.k, max_len, out=out)
+            X.score_topk_ex(q_fp8, w, ix.k_cache, ix.k_scale_cache, lengths, case.causal, case.k, max_len, out=out)
 
     def topk_only():
         X.topk(sc_view, lengths, case.causal, case.k, max_len, out=out)
@@ -209,7 +214,11 @@ def run_ours(args, rank, world, local_rank):
     def step():
         graph.replay()
 
-    X.quant_queries_append(q, w_raw, k_new, positions, ix.k_cache, ix.k_scale_cache, case.fmt, q_fp8, w)
+    if e8m0:
+        X.quant_queries(q, w_raw, case.fmt, q_fp8, w)
+        X.quant_append_e8(k_new, positions, ix.k_cache, ix.k_scale_cache)
+    else:
+        X.quant_queries_append(q, w_raw, k_new, positions, ix.k_cache, ix.k_scale_cache, case.fmt, q_fp8, w)
     for _ in range(args.warmup):
         step()
         score_only()
@@ -302,9 +311,9 @@ def run_ours(args, rank, world, local_rank):
     if topk_ms is not None:
         topk_ms = max_over_ranks([topk_ms], device=dev)[0]
     topk_bytes = B * n * 4 * (max_len + case.k) if ws_bytes else None   # score rows read, indices written
-    return dict(case=case, keys=keys, flops=flops, key_rows=key_rows, score_bytes=score_bytes, ms=ms,
+    return dict(case=case, e8m0=e8m0, keys=keys, flops=flops, key_rows=key_rows, score_bytes=score_bytes, ms=ms,
                 score_ms=score_ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
-                clocks=sampler.summary(), launches=(3 if ws_bytes else 2) * args.steps, topk_ms=topk_ms,
+                clocks=sampler.summary(), launches=(3 if (ws_bytes or e8m0) else 2) * args.steps, topk_ms=topk_ms,
                 topk_bytes=topk_bytes, two_pass=bool(ws_bytes))
 
 
@@ -408,6 +417,9 @@ def main():
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--scale-storage", choices=["f32", "e8m0"], default="f32",
+                    help="key scales as float32 (the workloads' layout) or one e8m0 byte per key "
+                         "(ue8m0 workloads only)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local_rank = env_rank()
@@ -452,7 +464,8 @@ def main():
                 "kernel_us": r["score_ms"] * 1e3, "algorithmic_flops": r["flops"]}
     else:
         achieved = r["score_bytes"] / score_s / 1e9
-        traffic = profile_traffic(PROFILE_SCORE, r["key_rows"]) if args.workload == DEFAULT_WORKLOAD else None
+        traffic = (profile_traffic(PROFILE_SCORE, r["key_rows"])
+                   if args.workload == DEFAULT_WORKLOAD and not r["e8m0"] else None)
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": traffic, "peak_source": f"{peak_src} copy bandwidth",
                 "kernel": "score (tcgen05 FP8 scorer, fp32 scores to the workspace)" if r["two_pass"]
@@ -462,9 +475,12 @@ def main():
         "metric": metric_name(case), "value": value, "unit": "keys/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8-e4m3 x fp8-e4m3 -> fp32", "data": "synthetic",
-        "config": {"workload": case.name, "B": case.B, "n": case.n, "T_cap": case.T_cap, "k": case.k,
+        "config": {"workload": case.name + (", e8m0 scale bytes" if r["e8m0"] else ""), "B": case.B, "n": case.n,
+                   "T_cap": case.T_cap, "k": case.k,
+                   "scale_storage": "e8m0 bytes (129 B/key)" if r["e8m0"] else "fp32 (132 B/key)",
                    "heads": 64, "head_dim": 128, "fmt": ["fp32", "ue8m0"][case.fmt],
-                   "l2": ("inputs larger than L2: %.0f MB FP8 cache streamed per step" % (r["key_rows"] * KEY_BYTES / 1e6))
+                   "l2": ("inputs larger than L2: %.0f MB FP8 cache streamed per step"
+                          % (r["key_rows"] * (KEY_BYTES - 3 * r["e8m0"]) / 1e6))
                    if r["key_rows"] * KEY_BYTES > 126e6 else "L2-resident working set (not flushed)",
                    "parallelism": f"dp{world} (independent sequences per rank)"},
         "roofline": roof,

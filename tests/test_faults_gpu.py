@@ -71,3 +71,44 @@ def test_bounded_wait_expires_cleanly():
     idx = X.score_topk(qc, w, kc, ks, lengths, False, 64, 1001)
     assert X.status() == (0, 0)
     assert np.all(idx.cpu().numpy() >= 0)
+
+
+def _prefill():
+    from tests.helpers import gpu_queries, gpu_state
+    case = synth.make_case("fault-prefill", 77, 2, 130, [200, 900], T_cap=2048, causal=True, fmt=1, k=64)
+    kc, ks, lengths = gpu_state(case)
+    qc, w = gpu_queries(case)
+    return case, kc, ks, lengths, qc, w
+
+
+def test_prefill_route_bounded_wait_expires_cleanly():
+    """The workspace route (flat-partition scorer, then the top-k kernel): a
+    scorer CTA that gives up reports a timeout; the next call is served."""
+    from sparse_attention_token_idx_b200 import binding as X
+    case, kc, ks, lengths, qc, w = _prefill()
+    max_len = int(case.lengths.max())
+    ws = torch.empty(X.workspace_size(2, 130, max_len, 64), dtype=torch.uint8, device="cuda")
+    try:
+        X.debug_set(1, 20_000_000)
+        X.score_topk(qc, w, kc, ks, lengths, True, 64, max_len, ws=ws)
+        code, bits = X.status()
+        assert code == -7 and bits & X.DEV_ERR_TIMEOUT
+    finally:
+        X.debug_set(0, 0)
+    idx = X.score_topk(qc, w, kc, ks, lengths, True, 64, max_len, ws=ws)
+    ref = X.score_topk(qc, w, kc, ks, lengths, True, 64, max_len)          # the single-kernel path
+    assert X.status() == (0, 0)
+    assert torch.equal(torch.sort(idx, -1).values, torch.sort(ref, -1).values)
+
+
+def test_prefill_route_lengths_beyond_max_len_are_reported_and_rows_emptied():
+    from sparse_attention_token_idx_b200 import binding as X
+    case, kc, ks, lengths, qc, w = _prefill()
+    max_len = 400                                    # sequence 1 has 1030 keys
+    ws = torch.empty(X.workspace_size(2, 130, max_len, 64), dtype=torch.uint8, device="cuda")
+    idx = X.score_topk(qc, w, kc, ks, lengths, True, 64, max_len, ws=ws).cpu().numpy()
+    code, bits = X.status()
+    assert code == -7 and bits & X.DEV_ERR_LENGTH
+    assert np.all(idx[1] == -1)
+    assert np.all(idx[0, :, :64][idx[0, :, :64] >= 0] < 330)
+    assert X.status() == (0, 0)

@@ -52,3 +52,35 @@ def test_graph_replay_equals_eager_step():
     torch.cuda.synchronize()
     assert X.status() == (0, 0)
     np.testing.assert_array_equal(out.cpu().numpy(), eager.cpu().numpy())
+
+
+@pytest.mark.parametrize("n,positions,causal", [(1, [500, 3000, 16383, 1, 2047, 9000, 12000, 7], False),
+                                                (48, [0, 700, 4000, 100, 9000, 12, 16000, 300], True)])
+def test_e8m0_scale_storage_selects_the_same_sets(n, positions, causal):
+    """Indexer with one e8m0 byte per key (129 cache bytes per key) against the
+    fp32 ue8m0 cache, eager and through a CUDA graph."""
+    from sparse_attention_token_idx_b200.pipeline import Indexer
+    from sparse_attention_token_idx_b200 import binding as X
+    positions = [min(p, 16384 - n) for p in positions]
+    case = synth.make_case("e8", 520 + n, 8, n, positions, T_cap=16384, causal=causal, fmt=1, k=256)
+    args = (bf16_dev(case.k_new), bf16_dev(case.q), dev(case.w_raw), dev(case.positions), dev(case.lengths))
+    ixs = [Indexer(case.B, case.T_cap, 1, case.k), Indexer(case.B, case.T_cap, 1, case.k, scale_storage="e8m0")]
+    for b in range(case.B):
+        p = int(case.positions[b])
+        if p:
+            kp, z = bf16_dev(case.k_prior[b:b + 1, :p]), dev(np.zeros(1, np.int32))
+            X.quant_append(kp, z, ixs[0].k_cache[b:b + 1], ixs[0].k_scale_cache[b:b + 1], 1)
+            X.quant_append_e8(kp, z, ixs[1].k_cache[b:b + 1], ixs[1].k_scale_cache[b:b + 1])
+    max_len = int(case.lengths.max())
+    ref = ixs[0].step(*args, causal=causal, max_len=max_len).clone()
+    got = ixs[1].step(*args, causal=causal, max_len=max_len).clone()
+    g, out = ixs[1].capture(*args, causal=causal, max_len=max_len)
+    out.fill_(-7)
+    g.replay()
+    torch.cuda.synchronize()
+    assert X.status() == (0, 0)
+    assert ixs[1].k_scale_cache.dtype == torch.uint8
+    assert torch.equal(ixs[0].k_cache, ixs[1].k_cache)
+    srt = lambda t: torch.sort(t, -1).values.cpu().numpy()
+    np.testing.assert_array_equal(srt(got), srt(ref))
+    np.testing.assert_array_equal(srt(out), srt(ref))
