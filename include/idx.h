@@ -212,6 +212,53 @@ IDX_API int idx_topk(const float* scores, const int32_t* lengths, int B, int n, 
              int32_t* indices, void* ws, size_t ws_bytes, idx_stream_t stream);
 
 /*
+ * Split-T selection: one sequence's keys split over G GPUs (or G slices on one
+ * GPU).  The Indexer.forward excerpt selects the row's top min(index_topk, ·)
+ * and then checks with a broadcast that every rank agrees; here each rank
+ * selects the k best of its own slice (idx_topk on its scores), turns them into
+ * (score, global position) pairs with idx_gather_scores, the ranks exchange the
+ * pairs (one all-gather of k·8 bytes per row), and idx_merge_topk selects the
+ * row's k best among the G·k candidates.  Exact: a key of the row's top k is in
+ * its own slice's top k.
+ */
+typedef struct {
+  float score;   /* the key's score */
+  int32_t pos;   /* its position in the whole sequence; −1 marks an empty slot */
+} idx_cand_t;    /* 8 bytes */
+
+/*
+ * idx_gather_scores
+ *   scores [rows, ld] float32 (device): this slice's scores, row r at r·ld.
+ *   idx [rows, k] int32 (device): slice-local positions from idx_topk, −1 = empty.
+ *   counts [rows] int32 (device) or NULL: keys of row r held in this slice;
+ *          positions ≥ counts[r] count as empty.  (A slice holding none of a
+ *          row's keys is scored and selected with a length of 1 — the scorer
+ *          requires lengths ≥ n — and its one position is dropped here.)
+ *   offset: the slice's first global position (added to every valid position).
+ *   cand [rows, k] idx_cand_t (device, caller-owned, 8-byte aligned) out:
+ *   (scores[r·ld + idx], idx + offset); empty slots give (−inf, −1).
+ *   Errors: IDX_ERR_SHAPE (rows, k < 0 or ld ≤ 0), IDX_ERR_NULL; nothing to do
+ *   when rows·k = 0.
+ */
+IDX_API int idx_gather_scores(const float* scores, int64_t ld, const int32_t* idx, int64_t rows, int k,
+                              const int32_t* counts, int32_t offset, idx_cand_t* cand, idx_stream_t stream);
+
+/*
+ * idx_merge_topk
+ *   cand [G, rows, kin] idx_cand_t (device): rank g's candidates of row r at
+ *   (g·rows + r)·kin — the layout of an all-gather of the per-rank [rows, kin]
+ *   outputs of idx_gather_scores.  Empty slots (pos −1) are skipped; the others
+ *   need finite scores and distinct positions.
+ *   out [rows, k] int32 (device, caller-owned): the positions of the
+ *   k_t = min(k, valid candidates) highest scores in columns 0 … k_t−1 (a set,
+ *   ties at the k_t-th score broken arbitrarily), −1 after.
+ *   Limits: G·kin ≤ 16384.  Errors: IDX_ERR_SHAPE, IDX_ERR_K (k ≤ 0), IDX_ERR_NULL.
+ *   One CTA per row.
+ */
+IDX_API int idx_merge_topk(const idx_cand_t* cand, int G, int64_t rows, int kin, int k, int32_t* out,
+                           idx_stream_t stream);
+
+/*
  * idx_score_topk — scores and top-k in one call, arguments as in idx_score /
  * idx_topk.  Decode-shaped calls (n ≤ 2) run one kernel in which a row's scores
  * never leave on-chip memory.  Prefill-shaped calls (n > 2) given a workspace of

@@ -45,6 +45,8 @@ SIGNATURES = {
     "idx_score_visible": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P]),
     "idx_score_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _P, _I64, _I, ctypes.c_float, _P]),
     "idx_topk": (_I, [_P, _P, _I, _I, _I64, _I, _I, _I, _P, _P, _SZ, _P]),
+    "idx_gather_scores": (_I, [_P, _I64, _P, _I64, _I, _P, _I, _P, _P]),
+    "idx_merge_topk": (_I, [_P, _I, _I64, _I, _I, _P, _P]),
     "idx_score_topk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "idx_score_topk_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
     "idx_score_topk_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
@@ -227,6 +229,42 @@ def score_topk_ex(q_fp8, w, k_cache, k_scale, lengths, causal: bool, k: int, max
                                     _ptr(lengths, torch.int32, "lengths"), B, n, k_cache.shape[1], max_len,
                                     int(causal), k, _ptr(out, torch.int32, "indices"), wsp, wsn, _stream(stream)),
            "idx_score_topk_ex")
+    return out
+
+
+def gather_scores(scores, idx, offset: int, counts=None, out=None, stream=None):
+    """(score, global position) pairs of a slice's top-k: scores [rows, ld] fp32,
+    idx [rows, k] int32 slice-local (−1 empty), counts [rows] int32 keys held per
+    row (None: all) → int32 [rows, k, 2] holding idx_cand_t pairs (score bits,
+    position); (−inf, −1) for empty slots."""
+    rows, ld = scores.shape
+    k = idx.shape[-1]
+    if tuple(idx.shape) != (rows, k):
+        raise ValueError("gather_scores: scores [rows, ld], idx [rows, k]")
+    out = out if out is not None else torch.empty((rows, k, 2), dtype=torch.int32, device=scores.device)
+    if tuple(out.shape[-3:]) != (rows, k, 2):
+        raise ValueError("gather_scores: out [rows, k, 2] int32")
+    _check(load().idx_gather_scores(_ptr(scores, torch.float32, "scores"), ld, _ptr(idx, torch.int32, "idx"), rows, k,
+                                    _ptr(counts, torch.int32, "counts"), int(offset), _ptr(out, torch.int32, "cand"),
+                                    _stream(stream)),
+           "idx_gather_scores")
+    return out
+
+
+def cand_scores(cand: torch.Tensor) -> torch.Tensor:
+    """The score plane of idx_cand_t pairs (int32 [..., 2]) as float32 [...]."""
+    return cand.view(torch.float32)[..., 0]
+
+
+def merge_topk(cand, k: int, out=None, stream=None):
+    """Top-k positions [rows, k] int32 among candidates int32 [G, rows, kin, 2]
+    (idx_cand_t pairs; position −1 = empty)."""
+    if cand.dim() != 4 or cand.shape[-1] != 2:
+        raise ValueError("merge_topk: cand int32 [G, rows, kin, 2]")
+    G, rows, kin, _ = cand.shape
+    out = out if out is not None else torch.empty((rows, k), dtype=torch.int32, device=cand.device)
+    _check(load().idx_merge_topk(_ptr(cand, torch.int32, "cand"), G, rows, kin, k, _ptr(out, torch.int32, "out"),
+                                 _stream(stream)), "idx_merge_topk")
     return out
 
 

@@ -298,6 +298,157 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(const RowParam
   if (tr && tid == 0) tr[4] = globaltimer_ns();
 }
 
+// ---------------------------------------------------------------------------
+// A sequence's keys split over G GPUs: each GPU selects the k best of its
+// slice and contributes them as (score, position) pairs; one exchange gives
+// every GPU all G·k candidates of a row, and the merge selects the row's k best
+// among them.  Exact: a key in the row's top k is in its own slice's top k.
+
+__global__ void __launch_bounds__(256) gather_scores_kernel(const float* __restrict__ scores, int64_t ld,
+                                                            const int32_t* __restrict__ idx, int64_t rows, int k,
+                                                            const int32_t* __restrict__ counts, int32_t offset,
+                                                            idx_cand_t* __restrict__ cand) {
+  const int64_t total = rows * k;
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = t / k;
+    const int32_t i0 = idx[t];
+    const int32_t i = (counts && i0 >= counts[r]) ? -1 : i0;
+    idx_cand_t c;
+    c.score = i >= 0 ? scores[r * ld + i] : -INFINITY;
+    c.pos = i >= 0 ? i + offset : -1;
+    cand[t] = c;
+  }
+}
+
+constexpr int kMergeMax = 16384;   // candidates per row (16-bit slots, one CTA)
+constexpr int kMergeThreads = 512;
+
+struct MergeLayout {
+  int hist1, cand, keys, pos, sel, total;
+};
+
+// shared memory: selection state | level-1 histogram | bin-b1 slot list |
+// order keys [m4] | positions [m4] | selected slots [m4]
+__host__ __device__ inline MergeLayout merge_layout(int m4, int cand_cap) {
+  MergeLayout l;
+  l.hist1 = (static_cast<int>(sizeof(CtaSelSmem)) + 127) / 128 * 128;
+  l.cand = l.hist1 + kHistBins * 4;
+  l.keys = l.cand + (cand_cap * 2 + 15) / 16 * 16;
+  l.pos = l.keys + m4 * 4;
+  l.sel = l.pos + m4 * 4;
+  l.total = l.sel + m4 * 4;
+  return l;
+}
+
+// One CTA per row.  Candidates [G, rows, kin] (rank-major, as an all-gather of
+// the per-GPU [rows, kin] arrays lays them out); slot s = g·kin + j of row r.
+// PAIRS2: kin even and cand 16-byte aligned, so two pairs come in one load.
+template <bool PAIRS2>
+__global__ void __launch_bounds__(kMergeThreads) merge_topk_kernel(const idx_cand_t* __restrict__ cand, int G,
+                                                                   int64_t rows, int kin, int k, int cand_cap,
+                                                                   int32_t* __restrict__ out) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
+  const int m = G * kin, m4 = (m + 3) & ~3;
+  const MergeLayout L = merge_layout(m4, cand_cap);
+  CtaSelSmem& sel = *reinterpret_cast<CtaSelSmem*>(smem);
+  uint32_t* hist1 = reinterpret_cast<uint32_t*>(smem + L.hist1);
+  uint16_t* cand16 = reinterpret_cast<uint16_t*>(smem + L.cand);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L.keys);
+  int32_t* pos_s = reinterpret_cast<int32_t*>(smem + L.pos);
+  int32_t* sel_s = reinterpret_cast<int32_t*>(smem + L.sel);
+  __shared__ int nvalid, next;
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int64_t row = blockIdx.x;
+  int32_t* o = out + row * k;
+  select_prepare(sel);
+  for (int t = tid; t < kHistBins; t += nthr) hist1[t] = 0u;
+  for (int t = m + tid; t < m4; t += nthr) keys[t] = 0u;
+  if (tid == 0) {
+    nvalid = 0;
+    next = 0;
+  }
+  __syncthreads();
+  int mine = 0;
+  // empty slots (position −1) get key 0: below every bin a score maps to
+  auto put = [&](int s, float score, int32_t p) {
+    const bool ok = p >= 0;
+    const uint32_t key = ok ? order_key(score) : 0u;
+    keys[s] = key;
+    pos_s[s] = p;
+    if (ok) {
+      select_count_key(sel, hist1, key);
+      ++mine;
+    }
+  };
+  constexpr int U = 4;   // loads in flight per thread
+  if (PAIRS2) {
+    const int half = kin >> 1, items = G * half;
+    for (int j0 = tid; j0 < items; j0 += U * nthr) {
+      int4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + u * nthr;
+        if (j < items) {
+          const int g = j / half, jj = j - g * half;
+          v[u] = __ldg(reinterpret_cast<const int4*>(cand + (static_cast<int64_t>(g) * rows + row) * kin) + jj);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + u * nthr;
+        if (j < items) {
+          const int g = j / half, s = g * kin + 2 * (j - g * half);
+          put(s, __int_as_float(v[u].x), v[u].y);
+          put(s + 1, __int_as_float(v[u].z), v[u].w);
+        }
+      }
+    }
+  } else {
+    for (int s0 = tid; s0 < m; s0 += U * nthr) {
+      int2 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int s = s0 + u * nthr;
+        if (s < m) {
+          const int g = s / kin;
+          v[u] = __ldg(reinterpret_cast<const int2*>(cand + (static_cast<int64_t>(g) * rows + row) * kin) +
+                       (s - g * kin));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int s = s0 + u * nthr;
+        if (s < m) put(s, __int_as_float(v[u].x), v[u].y);
+      }
+    }
+  }
+  for (int o2 = 16; o2 > 0; o2 >>= 1) mine += __shfl_xor_sync(0xFFFFFFFFu, mine, o2);
+  if ((tid & 31) == 0 && mine) atomicAdd(&nvalid, mine);
+  __syncthreads();
+  const int v = nvalid;
+  const int kt = min(k, v);
+  if (kt == v) {
+    // every candidate is kept: compact them in slot order (one shared counter per warp step)
+    for (int base = 0; base < m4; base += nthr) {
+      const int s = base + tid;
+      const bool take = s < m && keys[s] != 0u;
+      const uint32_t mk = __ballot_sync(0xFFFFFFFFu, take);
+      int at = 0;
+      if ((tid & 31) == 0 && mk) at = atomicAdd(&next, __popc(mk));
+      at = __shfl_sync(0xFFFFFFFFu, at, 0) + __popc(mk & lanemask_lt());
+      if (take) o[at] = pos_s[s];
+    }
+    for (int t = kt + tid; t < k; t += nthr) o[t] = -1;
+    return;
+  }
+  // slots of the kt best (into shared memory), then their positions
+  cta_select_row(sel, keys, m, 0, kt, hist1, true, nullptr, 0, cand16, cand_cap, sel_s, nullptr, nullptr, nullptr);
+  __syncthreads();
+  for (int t = tid; t < k; t += nthr) o[t] = t < kt ? pos_s[sel_s[t]] : -1;
+}
+
 int pow2_floor_i(int x) {
   int r = 1;
   while (r * 2 <= x) r *= 2;
@@ -379,5 +530,41 @@ extern "C" int idx_topk(const float* scores, const int32_t* lengths, int B, int 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaLaunchKernelEx(&cfg, topk_kernel, p);
+  return check_launch();
+}
+
+extern "C" int idx_gather_scores(const float* scores, int64_t ld, const int32_t* idx, int64_t rows, int k,
+                                 const int32_t* counts, int32_t offset, idx_cand_t* cand, idx_stream_t stream) {
+  if (rows < 0 || k < 0 || ld <= 0) return IDX_ERR_SHAPE;
+  if (rows == 0 || k == 0) return IDX_OK;
+  if (!scores || !idx || !cand) return IDX_ERR_NULL;
+  const int64_t total = rows * k;
+  const int64_t blocks = (total + 255) / 256;
+  const int grid = static_cast<int>(blocks < 148 * 16 ? blocks : 148 * 16);
+  gather_scores_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(scores, ld, idx, rows, k, counts,
+                                                                                 offset, cand);
+  return check_launch();
+}
+
+extern "C" int idx_merge_topk(const idx_cand_t* cand, int G, int64_t rows, int kin, int k, int32_t* out,
+                              idx_stream_t stream) {
+  if (G <= 0 || rows < 0 || kin <= 0) return IDX_ERR_SHAPE;
+  if (k <= 0) return IDX_ERR_K;
+  if (rows == 0) return IDX_OK;
+  if (!cand || !out) return IDX_ERR_NULL;
+  if (static_cast<int64_t>(G) * kin > kMergeMax || rows > 0x7FFFFFFF) return IDX_ERR_SHAPE;
+  const int m4 = (G * kin + 3) & ~3;
+  const int cand_cap = 2048;
+  const int smem = merge_layout(m4, cand_cap).total + 128;
+  const bool pairs2 = (kin % 2) == 0 && (reinterpret_cast<uintptr_t>(cand) & 15u) == 0;
+  auto kern = pairs2 ? merge_topk_kernel<true> : merge_topk_kernel<false>;
+  static int configured[2] = {-1, -1};
+  if (configured[pairs2] < smem) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return check_launch();
+    configured[pairs2] = smem;
+  }
+  kern<<<static_cast<unsigned>(rows), kMergeThreads, static_cast<size_t>(smem),
+         reinterpret_cast<cudaStream_t>(stream)>>>(cand, G, rows, kin, k, cand_cap, out);
   return check_launch();
 }

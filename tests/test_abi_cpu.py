@@ -58,6 +58,13 @@ def test_host_argument_checks_run_before_any_device_work():
     assert lib.idx_score_ex(p16, p16, p16, p16, 0, p16, 1, 1, 16, 16, 0, p16, 16, 0, float("nan"), None) == -2
     assert lib.idx_score_topk_ex(p16, p16, p16, p16, 3, p16, 1, 1, 16, 16, 0, 8, p16, None, 0, None) == -3
     assert lib.idx_quant_append_e8(None, None, 1, 1, None, None, 16, None) == -1
+    # split-T calls
+    assert lib.idx_gather_scores(None, 0, None, 1, 1, None, 0, None, None) == -2      # ld ≤ 0
+    assert lib.idx_gather_scores(None, 16, None, 1, 1, None, 0, None, None) == -1
+    assert lib.idx_gather_scores(None, 16, None, 0, 5, None, 0, None, None) == 0      # nothing to do
+    assert lib.idx_merge_topk(None, 1, 1, 4, 0, None, None) == -4
+    assert lib.idx_merge_topk(p16, 8, 1, 4096, 16, p16, None) == -2                  # G·kin > 16384
+    assert lib.idx_merge_topk(None, 2, 1, 4, 4, None, None) == -1
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")

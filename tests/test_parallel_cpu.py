@@ -73,3 +73,99 @@ def test_two_gloo_ranks_shard_and_reduce():
     assert all(r[3] == (3, 1, 16) for r in res)
     assert all(r[4] == [1.5, 10.0] for r in res)          # max over ranks, element-wise
     assert all(r[5] == 6 for r in res)
+
+
+# ---------------------------------------------------------------------------- split-T
+from sparse_attention_token_idx_b200.parallel import exchange_candidates, key_slice, slice_counts  # noqa: E402
+
+
+def test_key_slice_covers_every_position_once():
+    for T in [0, 1, 127, 128, 1000, 65536]:
+        for world in [1, 2, 3, 8]:
+            seen = []
+            for r in range(world):
+                lo, hi = key_slice(T, r, world)
+                assert lo % 128 == 0 or lo == T
+                seen.extend(range(lo, hi))
+            assert seen == list(range(T))
+    with pytest.raises(ValueError):
+        key_slice(128, 1, 1)
+
+
+def test_slice_counts_add_up_to_the_lengths():
+    import torch
+    L = np.array([0, 1, 200, 511, 512, 513, 1000], np.int32)
+    tot = np.zeros_like(L)
+    for r in range(3):
+        lo, hi = key_slice(1024, r, 3)
+        c = slice_counts(L, lo, hi)
+        assert c.dtype == np.int32 and np.all((c >= 0) & (c <= hi - lo))
+        assert np.array_equal(slice_counts(torch.from_numpy(L), lo, hi).numpy(), c)
+        tot += c
+    assert np.array_equal(tot, np.minimum(L, 1024))
+
+
+def _split_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import torch
+        from oracle import indexer as O
+        from sparse_attention_token_idx_b200 import synth
+        T, k = 1024, 48
+        # two sequences: one reaching into every slice, one ending inside rank 0's slice
+        case = synth.make_case("split", 91, 2, 1, [900, 300], T_cap=T, k=k)
+        kc = np.zeros((case.B, T, 128), np.uint8)
+        ks = np.zeros((case.B, T), np.float32)
+        for b in range(case.B):
+            p = int(case.positions[b])
+            O.quant_append(case.k_prior[b:b + 1, :p], [0], kc[b:b + 1], ks[b:b + 1], 0)
+        O.quant_append(case.k_new, case.positions, kc, ks, 0)
+        qc, _, w = O.quant_queries(case.q, case.w_raw, 0)
+
+        def candidates(r):   # rank r's slice top-k as (score bits, global position) pairs
+            lo, hi = key_slice(T, r, world)
+            cnt = slice_counts(case.lengths, lo, hi)
+            S, _ = O.index_scores(qc, w, kc[:, lo:hi], ks[:, lo:hi], cnt, False, ncols=hi - lo, with_bound=False)
+            c = np.zeros((case.B, k, 2), np.int32)
+            for b in range(case.B):
+                t = O.topk_row(S[b, 0], int(cnt[b]), k)
+                ok = t >= 0
+                c[b, :, 0] = np.where(ok, S[b, 0][np.maximum(t, 0)], -np.inf).astype(np.float32).view(np.int32)
+                c[b, :, 1] = np.where(ok, t + lo, -1)
+            return c
+
+        got = exchange_candidates(torch.from_numpy(candidates(rank))).numpy()
+        expect = np.stack([candidates(r) for r in range(world)])
+        S, _ = O.index_scores(qc, w, kc, ks, case.lengths, False, with_bound=False)
+        merged_ok = []
+        for b in range(case.B):
+            cs = got[:, b, :, 0].reshape(-1).view(np.float32).astype(np.float64)
+            cp = got[:, b, :, 1].reshape(-1)
+            valid = cp >= 0
+            full = O.topk_row(S[b, 0], int(case.lengths[b]), k)
+            pick = O.topk_row(cs[valid], int(valid.sum()), k)
+            merged = cp[valid][pick[pick >= 0]]
+            merged_ok.append(set(merged.tolist()) == set(full[full >= 0].tolist()))
+        q.put((rank, bool(np.array_equal(got, expect)), merged_ok))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_split_t_exchange_and_merge():
+    """The all-gather lays candidates out rank-major, and the k best of the
+    union of slice top-ks are the whole sequence's top-k (oracle scores)."""
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_split_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(r[1] for r in res), "exchanged candidates are not in rank order"
+    assert all(all(r[2]) for r in res), "merged slice top-ks differ from the full top-k"
