@@ -28,6 +28,10 @@ What it computes, step by step, with the passage each step follows:
 * ``topk``             — ``Indexer.forward`` excerpt (top min(index_topk, ·)
   positions per row) and the NKI "DeepSeek-V3.2 Sparse Indexer Kernel API
   Reference" page, Notes and return types (int32, an unordered set).
+* ``layer_norm_bf16``, ``rope_bf16``, ``front`` — the steps before the
+  rotation in the ``Indexer.forward`` excerpt: the key LayerNorm (k_norm), and
+  the rotary embedding, not interleaved, of the queries and keys (gain and
+  bias in fp32, cos / sin tables per token: NKI page, parameters).
 * ``e8m0_encode`` / ``e8m0_decode`` — the power-of-two key scale stored as one
   byte, the "e8m0" of the ``fp8_index`` docstring ("Index scores" page).
 * ``MASK_BOUND_BF16``, ``scores_bf16`` — the NKI page's Notes: masked slots
@@ -55,6 +59,13 @@ Readings taken where the pages are silent (each one also listed in the design doc):
   negative finite bfloat16, −(2 − 2^−7) · 2^127 — exact in bf16 and fp32, so
   a bf16 consumer reads it unchanged.
 * A bf16 score is the round-to-nearest-even of the fp32 score.
+* RoPE turns the leading 64 features ("64 rotary" features of the query
+  heads, "Join query parts" page); not interleaved means feature i pairs with
+  i + 32.  The angles come in as cos / sin tables (NKI page), so the YaRN
+  frequency schedule is outside this step.
+* LayerNorm: biased variance, eps added under the square root, all in float64
+  with sums taken from feature 0 to 127; its output is bf16 (the activations'
+  type), and so is the RoPE output.  eps is an argument (fp32).
 
 Precision: the FP8 dot products are computed exactly in float64 (every product
 of two e4m3 values is a multiple of 2^-18 below 2^17.7, so a 128-term sum needs
@@ -235,6 +246,57 @@ def quant_queries(q_bf16_bits, w_raw, fmt):
     """Queries [.., 64, 128] bf16 → (codes, per-head scale, folded weights)."""
     codes, q_scale = rotate_quant(q_bf16_bits, fmt)
     return codes, q_scale, fold_weights(w_raw, q_scale)
+
+
+# --------------------------------------------------------------------------- front end
+ROPE_DIM = 64      # leading features the rotary embedding turns (the 64 rotary features)
+
+
+def layer_norm_bf16(k_bf16_bits, gain, bias, eps):
+    """Key LayerNorm over the 128 features (Indexer.forward excerpt: the key
+    projection goes through k_norm before RoPE; NKI page: fp32 gain and bias).
+    float64 throughout: mean = (Σ x, summed from feature 0 to 127) / 128,
+    var = (Σ (x − mean)², same order) / 128, y = ((x − mean) / sqrt(var + eps))
+    · gain + bias, one rounding per operation, then round to bf16."""
+    x = bf16_bits_to_f64(k_bf16_bits)
+    mean = np.add.accumulate(x, axis=-1)[..., -1] / D
+    d = x - mean[..., None]
+    var = np.add.accumulate(d * d, axis=-1)[..., -1] / D
+    sd = np.sqrt(var + float(np.float32(eps)))
+    g = np.asarray(gain, np.float32).astype(np.float64)
+    b = np.asarray(bias, np.float32).astype(np.float64)
+    y = (d / sd[..., None]) * g + b
+    return f64_to_bf16_bits(bf16_round(y))
+
+
+def rope_bf16(x_bf16_bits, cos, sin):
+    """Rotary embedding of the leading 64 features, not interleaved
+    (Indexer.forward excerpt): feature i and feature i + 32 (i < 32) are the
+    two coordinates turned by angle θ_i, (a, b) → (a·cos θ_i − b·sin θ_i,
+    b·cos θ_i + a·sin θ_i); features 64 … 127 pass unchanged.  cos / sin
+    [..., 32] float32 (the NKI page's cos / sin tables, per token, broadcast
+    over leading axes).  float64 (the products are exact), then bf16."""
+    x = bf16_bits_to_f64(x_bf16_bits)
+    c = np.asarray(cos, np.float32).astype(np.float64)
+    s = np.asarray(sin, np.float32).astype(np.float64)
+    half = ROPE_DIM // 2
+    a, b = x[..., :half], x[..., half:ROPE_DIM]
+    y = x.copy()
+    y[..., :half] = a * c - b * s
+    y[..., half:ROPE_DIM] = b * c + a * s
+    return f64_to_bf16_bits(bf16_round(y))
+
+
+def front(q_proj_bits, k_proj_bits, cos, sin, gain, bias, eps):
+    """Query and key rows after the projections, ready for the rotation
+    (Indexer.forward excerpt, in its order): q [..., 64, 128] gets RoPE; k
+    [..., 128] gets the LayerNorm, then RoPE.  cos / sin [..., 32] per token.
+    Returns bf16 bits (q, k)."""
+    cos = np.asarray(cos, np.float32)
+    sin = np.asarray(sin, np.float32)
+    q = rope_bf16(q_proj_bits, cos[..., None, :], sin[..., None, :])
+    k = rope_bf16(layer_norm_bf16(k_proj_bits, gain, bias, eps), cos, sin)
+    return q, k
 
 
 # --------------------------------------------------------------------------- scores

@@ -511,3 +511,96 @@ def test_bf16_scores_match_torch_rounding():
     got = O.scores_bf16(x)
     fin = np.isfinite(want)
     assert np.array_equal(got[fin], want[fin])
+
+
+# --------------------------------------------------------------------------- front end
+def _bf16_bits(x):
+    return torch.from_numpy(np.asarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _bf16_vals(bits):
+    return torch.from_numpy(np.asarray(bits, np.uint16).view(np.int16)).view(torch.bfloat16).double().numpy()
+
+
+def test_rope_pairs_feature_i_with_i_plus_32():
+    """Non-interleaved pairing: a lone feature i < 32 moves only into i and
+    i + 32 (an interleaved or shifted pairing would light other slots)."""
+    th = np.linspace(0.1, 1.5, 32).astype(np.float32)
+    c, s = np.cos(th).astype(np.float32), np.sin(th).astype(np.float32)
+    for i in [0, 3, 31]:
+        x = np.zeros(128, np.float32)
+        x[i] = 1.0
+        y = _bf16_vals(O.rope_bf16(_bf16_bits(x), c, s))
+        assert set(np.flatnonzero(y)) == {i, i + 32}
+        assert y[i] == _bf16_vals(_bf16_bits([c[i]]))[0] and y[i + 32] == _bf16_vals(_bf16_bits([s[i]]))[0]
+        x = np.zeros(128, np.float32)
+        x[i + 32] = 1.0
+        y = _bf16_vals(O.rope_bf16(_bf16_bits(x), c, s))
+        assert set(np.flatnonzero(y)) == {i, i + 32}
+        assert y[i] == -_bf16_vals(_bf16_bits([s[i]]))[0]
+    x = np.zeros(128, np.float32)
+    x[64:] = np.arange(64) + 1
+    assert np.array_equal(O.rope_bf16(_bf16_bits(x), c, s), _bf16_bits(x))   # features 64 … 127 untouched
+
+
+def test_rope_special_angles_and_inverse():
+    rng = np.random.default_rng(4)
+    x = _bf16_bits(rng.standard_normal((6, 128)))
+    one, zero = np.ones(32, np.float32), np.zeros(32, np.float32)
+    assert np.array_equal(O.rope_bf16(x, one, zero), x)                   # θ = 0
+    v = _bf16_vals(x)
+    y = _bf16_vals(O.rope_bf16(x, zero, one))                            # θ = π/2: (a, b) → (−b, a)
+    assert np.array_equal(y[:, :32], -v[:, 32:64]) and np.array_equal(y[:, 32:64], v[:, :32])
+    # turning by θ and back stays within two bf16 roundings of the input
+    th = rng.uniform(-3, 3, 32)
+    f = O.rope_bf16(x, np.cos(th).astype(np.float32), np.sin(th).astype(np.float32))
+    back = _bf16_vals(O.rope_bf16(f, np.cos(-th).astype(np.float32), np.sin(-th).astype(np.float32)))
+    r = np.hypot(v[:, :32], v[:, 32:64])                                 # each pair's length
+    assert np.all(np.abs(back[:, :32] - v[:, :32]) <= 2 ** -7 * r)
+    assert np.all(np.abs(back[:, 32:64] - v[:, 32:64]) <= 2 ** -7 * r)
+    assert np.array_equal(back[:, 64:], v[:, 64:])
+
+
+def test_rope_matches_complex_multiplication():
+    """(a + i·b) · (cos θ + i·sin θ), numpy complex128, rounded to bf16."""
+    rng = np.random.default_rng(5)
+    x = _bf16_bits(rng.standard_normal((8, 128)) * 3)
+    th = rng.uniform(-np.pi, np.pi, (8, 32))
+    c, s = np.cos(th).astype(np.float32), np.sin(th).astype(np.float32)
+    v = _bf16_vals(x)
+    z = (v[:, :32] + 1j * v[:, 32:64]) * (c.astype(np.float64) + 1j * s.astype(np.float64))
+    want = v.copy()
+    want[:, :32], want[:, 32:64] = z.real, z.imag
+    want_bits = torch.from_numpy(want).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.rope_bf16(x, c, s), want_bits)
+
+
+def test_layer_norm_matches_torch_and_its_special_cases():
+    rng = np.random.default_rng(6)
+    x = _bf16_bits(rng.standard_normal((16, 128)) * rng.uniform(0.1, 30, (16, 1)) + rng.uniform(-5, 5, (16, 1)))
+    g = rng.uniform(0.5, 2, 128).astype(np.float32)
+    b = rng.uniform(-1, 1, 128).astype(np.float32)
+    eps = np.float32(1e-6)
+    ref = torch.nn.functional.layer_norm(torch.from_numpy(_bf16_vals(x)), (128,), torch.from_numpy(g).double(),
+                                         torch.from_numpy(b).double(), float(eps))
+    want = ref.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.layer_norm_bf16(x, g, b, eps), want)
+    # a constant row normalises to the bias; gain 1 / bias 0 gives mean 0 and variance 1
+    const = _bf16_bits(np.full((1, 128), 2.5))
+    assert np.array_equal(O.layer_norm_bf16(const, g, b, eps), _bf16_bits(b[None]))
+    y = _bf16_vals(O.layer_norm_bf16(x, np.ones(128, np.float32), np.zeros(128, np.float32), eps))
+    assert np.all(np.abs(y.mean(axis=1)) < 1e-2) and np.all(np.abs(y.var(axis=1) - 1) < 1e-2)
+
+
+def test_front_orders_layer_norm_before_rope_and_leaves_weights_alone():
+    rng = np.random.default_rng(7)
+    q = _bf16_bits(rng.standard_normal((2, 64, 128)))
+    k = _bf16_bits(rng.standard_normal((2, 128)) * 4 + 1)
+    th = rng.uniform(-3, 3, (2, 32))
+    c, s = np.cos(th).astype(np.float32), np.sin(th).astype(np.float32)
+    g, b = np.ones(128, np.float32), np.zeros(128, np.float32)
+    fq, fk = O.front(q, k, c, s, g, b, 1e-6)
+    for t in range(2):
+        assert np.array_equal(fq[t], O.rope_bf16(q[t], c[t], s[t]))
+    assert np.array_equal(fk, O.rope_bf16(O.layer_norm_bf16(k, g, b, 1e-6), c, s))
+    assert not np.array_equal(fk, O.layer_norm_bf16(O.rope_bf16(k, c, s), g, b, 1e-6))
