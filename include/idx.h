@@ -54,6 +54,7 @@ typedef struct CUstream_st* idx_stream_t;
 
 #define IDX_HEADS 64
 #define IDX_DIM 128
+#define IDX_ROPE_DIM 64    /* leading features the rotary embedding turns */
 #define IDX_MAX_LEN 131072 /* largest lengths[b] / max_len a score call accepts */
 
 enum idx_fmt { IDX_FMT_FP32 = 0, IDX_FMT_UE8M0 = 1 };
@@ -148,6 +149,35 @@ IDX_API int idx_quant_queries_append(const uint16_t* q_bf16, const float* w_raw,
                                      float* w, const uint16_t* k_bf16, const int32_t* positions, int B, int n,
                                      uint8_t* k_cache, float* k_scale_cache, int T_cap, int fmt,
                                      idx_stream_t stream);
+
+/*
+ * idx_front_quant_append — the indexer's front end after its projections, in
+ * the order of the Indexer.forward excerpt, fused with idx_quant_queries_append:
+ * queries get the rotary embedding; keys get the LayerNorm (k_norm), then the
+ * rotary embedding; both are then rotated and quantised, the keys appended and
+ * the weights folded as in idx_quant_queries_append.
+ *   q_proj [B, n, 64, 128] bf16: the query projection (wq_b of the low-rank
+ *          query), 16-byte aligned.
+ *   w_raw [B, n, 64] fp32: the weight projection of the hidden state.
+ *   k_proj [B, n, 128] bf16: the key projection (wk of the hidden state), 16-byte aligned.
+ *   rope_cos, rope_sin [B, n, IDX_ROPE_DIM / 2] fp32: cos θ_i and sin θ_i of
+ *          each token's position (the NKI page's cos / sin tables); feature
+ *          i and i + 32 (i < 32) are the pair turned by θ_i (not interleaved);
+ *          features 64 … 127 are not turned.
+ *   ln_gain, ln_bias [128] fp32, ln_eps ≥ 0: the key LayerNorm (biased
+ *          variance, eps under the square root).
+ *   positions, B, n, q_fp8, w, k_cache, k_scale_cache, T_cap, fmt: as in
+ *          idx_quant_queries_append (tokens = B·n).
+ * Arithmetic: float64 with one rounding per operation (sums over features in
+ * feature order), each step's result rounded to bf16, then the rotation and
+ * quantisation of idx_quant.  Errors as idx_quant_queries_append, plus
+ * IDX_ERR_SHAPE for a negative, infinite or NaN ln_eps.
+ */
+IDX_API int idx_front_quant_append(const uint16_t* q_proj, const float* w_raw, const uint16_t* k_proj,
+                                   const float* rope_cos, const float* rope_sin, const float* ln_gain,
+                                   const float* ln_bias, float ln_eps, const int32_t* positions, int B, int n,
+                                   uint8_t* q_fp8, float* w, uint8_t* k_cache, float* k_scale_cache, int T_cap,
+                                   int fmt, idx_stream_t stream);
 
 /*
  * idx_score — "Index scores" page: score equation and fp8_index docstring

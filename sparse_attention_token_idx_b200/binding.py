@@ -40,6 +40,8 @@ SIGNATURES = {
     "idx_quant_queries": (_I, [_P, _P, _I64, _P, _P, _I, _P]),
     "idx_quant_append": (_I, [_P, _P, _I, _I, _P, _P, _I, _I, _P]),
     "idx_quant_queries_append": (_I, [_P, _P, _I64, _P, _P, _P, _P, _I, _I, _P, _P, _I, _I, _P]),
+    "idx_front_quant_append": (_I, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _I, _I, _P, _P, _P, _P, _I, _I,
+                                    _P]),
     "idx_quant_append_e8": (_I, [_P, _P, _I, _I, _P, _P, _I, _P]),
     "idx_score": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P]),
     "idx_score_visible": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I64, _P]),
@@ -151,6 +153,28 @@ def quant_queries_append(q, w_raw, k_new, positions, k_cache, k_scale_cache, fmt
         _ptr(w_out, torch.float32, "w_out"), _ptr(k_new, _BF16, "k_new"), _ptr(positions, torch.int32, "positions"),
         B, n, _ptr(k_cache, torch.uint8, "k_cache"), _ptr(k_scale_cache, torch.float32, "k_scale_cache"),
         k_cache.shape[1], fmt, _stream(stream)), "idx_quant_queries_append")
+    return q_out, w_out
+
+
+def front_quant_append(q_proj, w_raw, k_proj, rope_cos, rope_sin, ln_gain, ln_bias, ln_eps: float, positions,
+                       k_cache, k_scale_cache, fmt, q_out=None, w_out=None, stream=None):
+    """Front end + quantisation in one launch: q_proj [B, n, 64, 128] bf16 gets
+    RoPE, k_proj [B, n, 128] bf16 gets LayerNorm then RoPE (cos / sin tables
+    [B, n, 32] fp32, gain / bias [128] fp32); then as quant_queries_append."""
+    B, n = k_proj.shape[0], k_proj.shape[1]
+    q_out = q_out if q_out is not None else torch.empty(tuple(q_proj.shape), dtype=torch.uint8, device=q_proj.device)
+    w_out = w_out if w_out is not None else torch.empty(tuple(w_raw.shape), dtype=torch.float32, device=q_proj.device)
+    if tuple(q_proj.shape) != (B, n, HEADS, DIM) or tuple(rope_cos.shape) != (B, n, 32) or \
+            tuple(rope_sin.shape) != (B, n, 32) or ln_gain.numel() != DIM or ln_bias.numel() != DIM:
+        raise ValueError("front_quant_append: q_proj [B, n, 64, 128], tables [B, n, 32], gain / bias [128]")
+    _check(load().idx_front_quant_append(
+        _ptr(q_proj, _BF16, "q_proj"), _ptr(w_raw, torch.float32, "w_raw"), _ptr(k_proj, _BF16, "k_proj"),
+        _ptr(rope_cos, torch.float32, "rope_cos"), _ptr(rope_sin, torch.float32, "rope_sin"),
+        _ptr(ln_gain, torch.float32, "ln_gain"), _ptr(ln_bias, torch.float32, "ln_bias"), float(ln_eps),
+        _ptr(positions, torch.int32, "positions"), B, n, _ptr(q_out, torch.uint8, "q_out"),
+        _ptr(w_out, torch.float32, "w_out"), _ptr(k_cache, torch.uint8, "k_cache"),
+        _ptr(k_scale_cache, torch.float32, "k_scale_cache"), k_cache.shape[1], fmt, _stream(stream)),
+        "idx_front_quant_append")
     return q_out, w_out
 
 

@@ -71,9 +71,7 @@ struct QuadRow {
   float scale;
 };
 
-__device__ __forceinline__ QuadRow rotate_quant_quad(const uint4* src, int fmt) {
-  const int q = threadIdx.x & 3;
-  double v[32];
+__device__ __forceinline__ void load_quad(const uint4* src, double (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint4 a = src[i];
@@ -84,6 +82,79 @@ __device__ __forceinline__ QuadRow rotate_quant_quad(const uint4* src, int fmt) 
       v[8 * i + 2 * m + 1] = bf16_to_f32(w[m] >> 16);
     }
   }
+}
+
+// Sum of the row's 128 values in feature order (0, 1, …, 127), float64: lane q
+// continues the running sum of lane q − 1.  All 32 lanes of the warp call it.
+__device__ __forceinline__ double quad_sequential_sum(const double (&v)[32]) {
+  const int lane = threadIdx.x & 31, q = lane & 3;
+  double acc = 0.0;
+#pragma unroll
+  for (int st = 0; st < 4; ++st) {
+    if (q == st) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) acc = __dadd_rn(acc, v[e]);
+    }
+    acc = __shfl_sync(0xFFFFFFFFu, acc, (lane & ~3) | st);
+  }
+  return acc;
+}
+
+__device__ __forceinline__ double bf16_round_f64(double x) { return static_cast<double>(f64_to_bf16_as_f32(x)); }
+
+// Key LayerNorm over the row (Indexer.forward excerpt: k_norm after the key
+// projection): mean and biased variance by feature-order sums, then
+// ((x − mean) / sqrt(var + eps)) · gain + bias, float64 with one rounding per
+// operation, then bf16.  All lanes call it; `apply` selects whose row changes.
+__device__ __forceinline__ void quad_layer_norm(double (&v)[32], bool apply, const float* __restrict__ gain,
+                                                const float* __restrict__ bias, double eps) {
+  const int q = threadIdx.x & 3;
+  const double mean = __dmul_rn(quad_sequential_sum(v), 0.0078125);
+  double d[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) d[e] = __dsub_rn(v[e], mean);
+  double sq[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) sq[e] = __dmul_rn(d[e], d[e]);
+  const double var = __dmul_rn(quad_sequential_sum(sq), 0.0078125);
+  const double sd = __dsqrt_rn(__dadd_rn(var, eps));
+  if (apply) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const double g = __ldg(gain + 32 * q + e), b = __ldg(bias + 32 * q + e);
+      v[e] = bf16_round_f64(__dadd_rn(__dmul_rn(__ddiv_rn(d[e], sd), g), b));
+    }
+  }
+}
+
+// Rotary embedding of features 0 … 63, not interleaved (Indexer.forward
+// excerpt): feature i (lane 0) and i + 32 (lane 1) turn by angle θ_i,
+// (a, b) → (a cos − b sin, b cos + a sin); the products are exact in float64,
+// so each result is rounded once, then to bf16.  All lanes call it.
+__device__ __forceinline__ void quad_rope(double (&v)[32], const float* __restrict__ cos_row,
+                                          const float* __restrict__ sin_row) {
+  const int q = threadIdx.x & 3;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const double o = __shfl_xor_sync(0xFFFFFFFFu, v[e], 1);
+    if (q < 2) {
+      const double c = __ldg(cos_row + e), s = __ldg(sin_row + e);
+      const double vc = __dmul_rn(v[e], c), os = __dmul_rn(o, s);
+      v[e] = bf16_round_f64(q == 0 ? __dsub_rn(vc, os) : __dadd_rn(vc, os));
+    }
+  }
+}
+
+__device__ __forceinline__ QuadRow rotate_quant_v(double (&v)[32], int fmt);
+
+__device__ __forceinline__ QuadRow rotate_quant_quad(const uint4* src, int fmt) {
+  double v[32];
+  load_quad(src, v);
+  return rotate_quant_v(v, fmt);
+}
+
+__device__ __forceinline__ QuadRow rotate_quant_v(double (&v)[32], int fmt) {
+  const int q = threadIdx.x & 3;
 #pragma unroll
   for (int h = 1; h < 32; h <<= 1) {
 #pragma unroll
@@ -154,8 +225,16 @@ struct QuantArgs {
   int n, T_cap;
   int fmt;
   unsigned int* err;
+  // front end (FRONT kernels): per-token RoPE tables [tokens, 32] (tokens = the
+  // key rows, each with 64 query rows) and the key LayerNorm's gain / bias / eps
+  const float* rope_cos;
+  const float* rope_sin;
+  const float* ln_gain;
+  const float* ln_bias;
+  double ln_eps;
 };
 
+template <bool FRONT>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32) quant_kernel(const QuantArgs a) {
   const int lane = threadIdx.x & 31;
   const int q = lane & 3;
@@ -190,7 +269,18 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) quant_kernel(const QuantA
       src = a.rows > 0 ? a.x : a.k;
       dst = nullptr;
     }
-    const QuadRow out = rotate_quant_quad(reinterpret_cast<const uint4*>(src + 32 * q), a.fmt);
+    QuadRow out;
+    if constexpr (FRONT) {
+      double v[32];
+      load_quad(reinterpret_cast<const uint4*>(src + 32 * q), v);
+      // the row's token: key row kr, or query row r of token r / 64 (0 past the end)
+      const int64_t tok = is_key ? r - a.rows : (live ? r / IDX_HEADS : 0);
+      quad_layer_norm(v, is_key, a.ln_gain, a.ln_bias, a.ln_eps);
+      quad_rope(v, a.rope_cos + tok * (IDX_ROPE_DIM / 2), a.rope_sin + tok * (IDX_ROPE_DIM / 2));
+      out = rotate_quant_v(v, a.fmt);
+    } else {
+      out = rotate_quant_quad(reinterpret_cast<const uint4*>(src + 32 * q), a.fmt);
+    }
     if (store) {
       uint4* d = reinterpret_cast<uint4*>(dst + 32 * q);
       d[0] = out.codes[0];
@@ -225,10 +315,13 @@ int quant_grid(int64_t rows) {
   return static_cast<int>(blocks < cap ? blocks : cap);
 }
 
-int launch_quant(const QuantArgs& a, cudaStream_t stream) {
+int launch_quant(const QuantArgs& a, cudaStream_t stream, bool front = false) {
   const int64_t total = a.rows + a.k_rows;
   if (total == 0) return IDX_OK;
-  quant_kernel<<<quant_grid(total), kWarpsPerBlock * 32, 0, stream>>>(a);
+  if (front)
+    quant_kernel<true><<<quant_grid(total), kWarpsPerBlock * 32, 0, stream>>>(a);
+  else
+    quant_kernel<false><<<quant_grid(total), kWarpsPerBlock * 32, 0, stream>>>(a);
   return check_launch();
 }
 
@@ -325,6 +418,46 @@ extern "C" int idx_quant_append_e8(const uint16_t* k_bf16, const int32_t* positi
   a.err = device_error_word();
   if (!a.err) return check_launch();
   return launch_quant(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int idx_front_quant_append(const uint16_t* q_proj, const float* w_raw, const uint16_t* k_proj,
+                                      const float* rope_cos, const float* rope_sin, const float* ln_gain,
+                                      const float* ln_bias, float ln_eps, const int32_t* positions, int B, int n,
+                                      uint8_t* q_fp8, float* w, uint8_t* k_cache, float* k_scale_cache, int T_cap,
+                                      int fmt, idx_stream_t stream) {
+  if (B < 0 || n < 0 || T_cap <= 0) return IDX_ERR_SHAPE;
+  if (fmt != IDX_FMT_FP32 && fmt != IDX_FMT_UE8M0) return IDX_ERR_FMT;
+  if (!(ln_eps >= 0.0f) || ln_eps > 3.0e38f) return IDX_ERR_SHAPE;   // NaN, negative or infinite
+  if (B == 0 || n == 0) return IDX_OK;
+  if (n > T_cap) return IDX_ERR_SHAPE;
+  if (!q_proj || !w_raw || !k_proj || !rope_cos || !rope_sin || !ln_gain || !ln_bias || !positions || !q_fp8 || !w ||
+      !k_cache || !k_scale_cache)
+    return IDX_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(q_proj) | reinterpret_cast<uintptr_t>(q_fp8) | reinterpret_cast<uintptr_t>(k_proj) |
+       reinterpret_cast<uintptr_t>(k_cache)) & 15)
+    return IDX_ERR_ALIGN;
+  const int64_t tokens = static_cast<int64_t>(B) * n;
+  QuantArgs a = empty_args(fmt);
+  a.x = q_proj;
+  a.codes = q_fp8;
+  a.w_raw = w_raw;
+  a.w_out = w;
+  a.rows = tokens * IDX_HEADS;
+  a.k = k_proj;
+  a.positions = positions;
+  a.k_cache = k_cache;
+  a.k_scale_cache = k_scale_cache;
+  a.k_rows = tokens;
+  a.n = n;
+  a.T_cap = T_cap;
+  a.rope_cos = rope_cos;
+  a.rope_sin = rope_sin;
+  a.ln_gain = ln_gain;
+  a.ln_bias = ln_bias;
+  a.ln_eps = static_cast<double>(ln_eps);
+  a.err = device_error_word();
+  if (!a.err) return check_launch();
+  return launch_quant(a, reinterpret_cast<cudaStream_t>(stream), true);
 }
 
 extern "C" int idx_e4m3_encode(const float* x, int64_t count, uint8_t* out, idx_stream_t stream) {

@@ -65,6 +65,26 @@ class Indexer:
         return X.score_topk_ex(q_fp8, w, self.k_cache, self.k_scale_cache, lengths, causal, self.k, max_len,
                                out=out, ws=ws, stream=stream)
 
+    def step_front(self, q_proj, w_raw, k_proj, rope_cos, rope_sin, ln_gain, ln_bias, positions, lengths, *,
+                   causal: bool, max_len: int, ln_eps: float = 1e-6, out=None, stream=None):
+        """One indexer call from the projections on (the caller's GEMMs: q_proj =
+        wq_b(qr) [B, n, 64, 128] bf16, k_proj = wk(x) [B, n, 128] bf16, w_raw =
+        weights_proj(x) [B, n, 64] fp32): query RoPE, key LayerNorm + RoPE,
+        rotation, quantisation and append in one launch, then score + top-k.
+        fp32 scale storage only."""
+        if self.e8m0:
+            raise ValueError("step_front writes fp32 key scales")
+        B, n = k_proj.shape[0], k_proj.shape[1]
+        q_fp8 = self._buf("q_fp8", tuple(q_proj.shape), torch.uint8)
+        w = self._buf("w", tuple(w_raw.shape), torch.float32)
+        X.front_quant_append(q_proj, w_raw, k_proj, rope_cos, rope_sin, ln_gain, ln_bias, ln_eps, positions,
+                             self.k_cache, self.k_scale_cache, self.fmt, q_fp8, w, stream=stream)
+        out = out if out is not None else self._buf("idx", (B, n, self.k), torch.int32)
+        ws_bytes = X.workspace_size(B, n, max_len, self.k)
+        ws = self._buf("ws", (ws_bytes,), torch.uint8) if ws_bytes else None
+        return X.score_topk_ex(q_fp8, w, self.k_cache, self.k_scale_cache, lengths, causal, self.k, max_len,
+                               out=out, ws=ws, stream=stream)
+
     def capture(self, k_new, q, w_raw, positions, lengths, *, causal: bool, max_len: int):
         """Record one step on static input tensors into a CUDA graph; returns
         (graph, out) — replay the graph after refilling the inputs in place."""

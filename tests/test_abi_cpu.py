@@ -58,6 +58,15 @@ def test_host_argument_checks_run_before_any_device_work():
     assert lib.idx_score_ex(p16, p16, p16, p16, 0, p16, 1, 1, 16, 16, 0, p16, 16, 0, float("nan"), None) == -2
     assert lib.idx_score_topk_ex(p16, p16, p16, p16, 3, p16, 1, 1, 16, 16, 0, 8, p16, None, 0, None) == -3
     assert lib.idx_quant_append_e8(None, None, 1, 1, None, None, 16, None) == -1
+    # front end: unknown fmt, bad eps, nothing to do, a missing table
+    assert lib.idx_front_quant_append(p16, p16, p16, p16, p16, p16, p16, 1e-6, p16, 1, 1, p16, p16, p16, p16, 16, 7,
+                                      None) == -3
+    assert lib.idx_front_quant_append(p16, p16, p16, p16, p16, p16, p16, float("nan"), p16, 1, 1, p16, p16, p16, p16,
+                                      16, 0, None) == -2
+    assert lib.idx_front_quant_append(None, None, None, None, None, None, None, 1e-6, None, 0, 1, None, None, None,
+                                      None, 16, 0, None) == 0
+    assert lib.idx_front_quant_append(p16, p16, p16, None, p16, p16, p16, 1e-6, p16, 1, 1, p16, p16, p16, p16, 16, 0,
+                                      None) == -1
     # split-T calls
     assert lib.idx_gather_scores(None, 0, None, 1, 1, None, 0, None, None) == -2      # ld ≤ 0
     assert lib.idx_gather_scores(None, 16, None, 1, 1, None, 0, None, None) == -1
