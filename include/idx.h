@@ -289,6 +289,27 @@ IDX_API int idx_merge_topk(const idx_cand_t* cand, int G, int64_t rows, int kin,
                            idx_stream_t stream);
 
 /*
+ * idx_sparse_mla_decode — the attention that consumes the selection ("Join
+ * query parts" page, MQA decode excerpt): for one decode token per sequence,
+ * each head scores the selected cache rows, takes the softmax over them and
+ * returns the latent output.
+ *   q [B, H, 576] bf16: per head the absorbed content query (512) followed by
+ *          the rotary query (64); H a multiple of 16.
+ *   kv [B, T_cap, 576] bf16 (16-byte aligned): per position the latent (512)
+ *          followed by the rotary key (64).
+ *   indices [B, k] int32: the selected positions (the indexer's output for the
+ *          token); entries < 0 or ≥ T_cap select nothing.
+ *   softmax_scale: finite; s = softmax_scale · q·kv.
+ *   out [B, H, 512] fp32 (caller-owned): Σ_t softmax(s)_t · kv[t, 0:512]
+ *          over the selected t; 0 for a row that selects nothing.
+ * Arithmetic: fp32 on the CUDA cores (online softmax over chunks of 32
+ * positions).  Errors: IDX_ERR_SHAPE (B < 0, H not a positive multiple of 16,
+ * T_cap ≤ 0, a non-finite scale), IDX_ERR_K (k ≤ 0), IDX_ERR_NULL, IDX_ERR_ALIGN.
+ */
+IDX_API int idx_sparse_mla_decode(const uint16_t* q, const uint16_t* kv, const int32_t* indices, int B, int H,
+                                  int64_t T_cap, int k, float softmax_scale, float* out, idx_stream_t stream);
+
+/*
  * idx_score_topk — scores and top-k in one call, arguments as in idx_score /
  * idx_topk.  Decode-shaped calls (n ≤ 2) run one kernel in which a row's scores
  * never leave on-chip memory.  Prefill-shaped calls (n > 2) given a workspace of

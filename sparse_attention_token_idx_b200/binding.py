@@ -49,6 +49,7 @@ SIGNATURES = {
     "idx_topk": (_I, [_P, _P, _I, _I, _I64, _I, _I, _I, _P, _P, _SZ, _P]),
     "idx_gather_scores": (_I, [_P, _I64, _P, _I64, _I, _P, _I, _P, _P]),
     "idx_merge_topk": (_I, [_P, _I, _I64, _I, _I, _P, _P]),
+    "idx_sparse_mla_decode": (_I, [_P, _P, _P, _I, _I, _I64, _I, ctypes.c_float, _P, _P]),
     "idx_score_topk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "idx_score_topk_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
     "idx_score_topk_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
@@ -289,6 +290,21 @@ def merge_topk(cand, k: int, out=None, stream=None):
     out = out if out is not None else torch.empty((rows, k), dtype=torch.int32, device=cand.device)
     _check(load().idx_merge_topk(_ptr(cand, torch.int32, "cand"), G, rows, kin, k, _ptr(out, torch.int32, "out"),
                                  _stream(stream)), "idx_merge_topk")
+    return out
+
+
+def sparse_mla_decode(q, kv, indices, softmax_scale: float, out=None, stream=None):
+    """Latent output [B, H, 512] fp32 of one decode token per sequence attending
+    over its selected positions: q [B, H, 576] bf16, kv [B, T_cap, 576] bf16,
+    indices [B, k] int32 (−1 = none)."""
+    B, H, D = q.shape
+    if D != 576 or kv.dim() != 3 or kv.shape[0] != B or kv.shape[2] != 576 or indices.dim() != 2 or \
+            indices.shape[0] != B:
+        raise ValueError("sparse_mla_decode: q [B, H, 576], kv [B, T_cap, 576], indices [B, k]")
+    out = out if out is not None else torch.empty((B, H, 512), dtype=torch.float32, device=q.device)
+    _check(load().idx_sparse_mla_decode(_ptr(q, _BF16, "q"), _ptr(kv, _BF16, "kv"), _ptr(indices, torch.int32, "indices"),
+                                        B, H, kv.shape[1], indices.shape[1], float(softmax_scale),
+                                        _ptr(out, torch.float32, "out"), _stream(stream)), "idx_sparse_mla_decode")
     return out
 
 

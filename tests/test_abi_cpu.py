@@ -67,6 +67,12 @@ def test_host_argument_checks_run_before_any_device_work():
                                       None, 16, 0, None) == 0
     assert lib.idx_front_quant_append(p16, p16, p16, None, p16, p16, p16, 1e-6, p16, 1, 1, p16, p16, p16, p16, 16, 0,
                                       None) == -1
+    # sparse latent attention: heads not a multiple of 16, k ≤ 0, a NaN scale, nothing to do, null
+    assert lib.idx_sparse_mla_decode(p16, p16, p16, 1, 24, 16, 8, 0.1, p16, None) == -2
+    assert lib.idx_sparse_mla_decode(p16, p16, p16, 1, 16, 16, 0, 0.1, p16, None) == -4
+    assert lib.idx_sparse_mla_decode(p16, p16, p16, 1, 16, 16, 8, float("nan"), p16, None) == -2
+    assert lib.idx_sparse_mla_decode(None, None, None, 0, 16, 16, 8, 0.1, None, None) == 0
+    assert lib.idx_sparse_mla_decode(p16, None, p16, 1, 16, 16, 8, 0.1, p16, None) == -1
     # split-T calls
     assert lib.idx_gather_scores(None, 0, None, 1, 1, None, 0, None, None) == -2      # ld ≤ 0
     assert lib.idx_gather_scores(None, 16, None, 1, 1, None, 0, None, None) == -1
