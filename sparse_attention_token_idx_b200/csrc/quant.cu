@@ -84,8 +84,10 @@ __device__ __forceinline__ void load_quad(const uint4* src, double (&v)[32]) {
   }
 }
 
-// Sum of the row's 128 values in feature order (0, 1, …, 127), float64: lane q
-// continues the running sum of lane q − 1.  All 32 lanes of the warp call it.
+// Sum of the row's 128 values (SQUARE: of their squares, each rounded) in
+// feature order (0, 1, …, 127), float64: lane q continues the running sum of
+// lane q − 1.  All 32 lanes of the warp call it.
+template <bool SQUARE>
 __device__ __forceinline__ double quad_sequential_sum(const double (&v)[32]) {
   const int lane = threadIdx.x & 31, q = lane & 3;
   double acc = 0.0;
@@ -93,7 +95,7 @@ __device__ __forceinline__ double quad_sequential_sum(const double (&v)[32]) {
   for (int st = 0; st < 4; ++st) {
     if (q == st) {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) acc = __dadd_rn(acc, v[e]);
+      for (int e = 0; e < 32; ++e) acc = __dadd_rn(acc, SQUARE ? __dmul_rn(v[e], v[e]) : v[e]);
     }
     acc = __shfl_sync(0xFFFFFFFFu, acc, (lane & ~3) | st);
   }
@@ -109,20 +111,19 @@ __device__ __forceinline__ double bf16_round_f64(double x) { return static_cast<
 __device__ __forceinline__ void quad_layer_norm(double (&v)[32], bool apply, const float* __restrict__ gain,
                                                 const float* __restrict__ bias, double eps) {
   const int q = threadIdx.x & 3;
-  const double mean = __dmul_rn(quad_sequential_sum(v), 0.0078125);
-  double d[32];
+  const double mean = __dmul_rn(quad_sequential_sum<false>(v), 0.0078125);
+  // rows that are not normalised keep their values (their statistics go unused)
+  if (apply) {
 #pragma unroll
-  for (int e = 0; e < 32; ++e) d[e] = __dsub_rn(v[e], mean);
-  double sq[32];
-#pragma unroll
-  for (int e = 0; e < 32; ++e) sq[e] = __dmul_rn(d[e], d[e]);
-  const double var = __dmul_rn(quad_sequential_sum(sq), 0.0078125);
+    for (int e = 0; e < 32; ++e) v[e] = __dsub_rn(v[e], mean);
+  }
+  const double var = __dmul_rn(quad_sequential_sum<true>(v), 0.0078125);
   const double sd = __dsqrt_rn(__dadd_rn(var, eps));
   if (apply) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const double g = __ldg(gain + 32 * q + e), b = __ldg(bias + 32 * q + e);
-      v[e] = bf16_round_f64(__dadd_rn(__dmul_rn(__ddiv_rn(d[e], sd), g), b));
+      v[e] = bf16_round_f64(__dadd_rn(__dmul_rn(__ddiv_rn(v[e], sd), g), b));
     }
   }
 }
@@ -275,7 +276,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) quant_kernel(const QuantA
       load_quad(reinterpret_cast<const uint4*>(src + 32 * q), v);
       // the row's token: key row kr, or query row r of token r / 64 (0 past the end)
       const int64_t tok = is_key ? r - a.rows : (live ? r / IDX_HEADS : 0);
-      quad_layer_norm(v, is_key, a.ln_gain, a.ln_bias, a.ln_eps);
+      // warps of query rows only skip the LayerNorm (warp-uniform: the shuffles stay converged)
+      if (__any_sync(0xFFFFFFFFu, is_key)) quad_layer_norm(v, is_key, a.ln_gain, a.ln_bias, a.ln_eps);
       quad_rope(v, a.rope_cos + tok * (IDX_ROPE_DIM / 2), a.rope_sin + tok * (IDX_ROPE_DIM / 2));
       out = rotate_quant_v(v, a.fmt);
     } else {
