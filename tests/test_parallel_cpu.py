@@ -169,3 +169,87 @@ def test_two_gloo_ranks_split_t_exchange_and_merge():
         assert p.exitcode == 0
     assert all(r[1] for r in res), "exchanged candidates are not in rank order"
     assert all(all(r[2]) for r in res), "merged slice top-ks differ from the full top-k"
+
+
+def _orchestration_worker(rank, world, port, q):
+    """split_t_decode on CPU tensors, the library calls replaced by stand-ins
+    computed with the oracle: the host logic (slice counts, the one-key
+    stand-in for empty slices, position offsets, the exchange) runs as is."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import torch
+        from oracle import indexer as O
+        from sparse_attention_token_idx_b200 import binding as X
+        from sparse_attention_token_idx_b200 import parallel as PL
+        from sparse_attention_token_idx_b200 import synth
+
+        def score_visible(q_fp8, w, kc, ks, lengths, causal, max_len, stream=None):
+            S, _ = O.index_scores(q_fp8.numpy(), w.numpy(), kc.numpy(), ks.numpy(), lengths.numpy(), causal,
+                                  ncols=max_len, with_bound=False)
+            return torch.from_numpy(S.astype(np.float32))
+
+        def topk(scores, lengths, causal, k, max_len, stream=None):
+            return torch.from_numpy(O.topk(scores.numpy().astype(np.float64), lengths.numpy(), causal, k))
+
+        def gather_scores(scores, idx, offset, counts=None, stream=None):
+            s, i = scores.numpy(), idx.numpy()
+            c = counts.numpy() if counts is not None else np.full(len(i), s.shape[1])
+            valid = (i >= 0) & (i < c[:, None])
+            out = np.zeros(i.shape + (2,), np.int32)
+            out[..., 0] = np.where(valid, np.take_along_axis(s, np.maximum(i, 0), 1), -np.inf).astype(
+                np.float32).view(np.int32)
+            out[..., 1] = np.where(valid, i + offset, -1)
+            return torch.from_numpy(out)
+
+        def merge_topk(cand, k, out=None, stream=None):
+            c = cand.numpy()
+            G, rows, kin, _ = c.shape
+            res = np.full((rows, k), -1, np.int32)
+            for r in range(rows):
+                sc = c[:, r, :, 0].reshape(-1).view(np.float32).astype(np.float64)
+                ps = c[:, r, :, 1].reshape(-1)
+                ok = ps >= 0
+                pick = O.topk_row(sc[ok], int(ok.sum()), k)
+                res[r, :(pick >= 0).sum()] = ps[ok][pick[pick >= 0]]
+            return torch.from_numpy(res)
+
+        X.score_visible, X.topk, X.gather_scores, X.merge_topk = score_visible, topk, gather_scores, merge_topk
+        T, k = 1024, 40
+        case = synth.make_case("split-orch", 93, 3, 1, [1000, 200, 600], T_cap=T, k=k)
+        kc = np.zeros((case.B, T, 128), np.uint8)
+        ks = np.zeros((case.B, T), np.float32)
+        for b in range(case.B):
+            p = int(case.positions[b])
+            O.quant_append(case.k_prior[b:b + 1, :p], [0], kc[b:b + 1], ks[b:b + 1], 0)
+        O.quant_append(case.k_new, case.positions, kc, ks, 0)
+        qc, _, w = O.quant_queries(case.q, case.w_raw, 0)
+        lo, hi = PL.key_slice(T, rank, world)
+        got = PL.split_t_decode(torch.from_numpy(qc), torch.from_numpy(w), torch.from_numpy(kc[:, lo:hi].copy()),
+                                torch.from_numpy(ks[:, lo:hi].copy()), torch.from_numpy(case.lengths), lo, hi,
+                                k).numpy()
+        S, _ = O.index_scores(qc, w, kc, ks, case.lengths, False, with_bound=False)
+        same = [set(got[b][got[b] >= 0].tolist()) == set(O.topk_row(S[b, 0], int(case.lengths[b]), k).tolist())
+                for b in range(case.B)]
+        q.put((rank, same, int((got >= 0).sum())))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_split_t_decode_orchestration():
+    """Rank 1 holds no key of the second sequence (length 201 < 512): its slice
+    is scored as one key and dropped; every rank ends with the full top-k."""
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_orchestration_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert all(all(r[1]) for r in res), "split-T result differs from the whole-sequence top-k"
+    assert all(r[2] == 3 * 40 for r in res)
