@@ -85,10 +85,12 @@ class Indexer:
         return X.score_topk_ex(q_fp8, w, self.k_cache, self.k_scale_cache, lengths, causal, self.k, max_len,
                                out=out, ws=ws, stream=stream)
 
-    def capture(self, k_new, q, w_raw, positions, lengths, *, causal: bool, max_len: int):
+    def capture(self, k_new, q, w_raw, positions, lengths, *, causal: bool, max_len: int, out=None):
         """Record one step on static input tensors into a CUDA graph; returns
-        (graph, out) — replay the graph after refilling the inputs in place."""
-        out = self._buf("idx_graph", (q.shape[0], q.shape[1], self.k), torch.int32)
+        (graph, out) — replay the graph after refilling the inputs in place.
+        The step also runs once, for real, before the capture (warm-up)."""
+        if out is None:
+            out = self._buf("idx_graph", (q.shape[0], q.shape[1], self.k), torch.int32)
         s = torch.cuda.Stream(device=self.device)
         s.wait_stream(torch.cuda.current_stream(self.device))
         with torch.cuda.stream(s):                      # warm-up outside the capture
@@ -98,3 +100,84 @@ class Indexer:
         with torch.cuda.graph(g):
             self.step(k_new, q, w_raw, positions, lengths, causal=causal, max_len=max_len, out=out)
         return g, out
+
+
+class HostPipeline:
+    """Indexer steps fed from pinned host memory with the copies overlapped.
+
+    A submitted step copies its inputs host → device on an upload stream,
+    replays its CUDA graph on the compute stream once they have landed, and
+    copies the top-k indices device → host on a download stream.  Two slots of
+    device buffers (each with its own graph) let step i+1's upload and step
+    i−1's download run while step i computes.  Steps compute in submission
+    order on one stream, so each sees the cache as the steps before it left it.
+    A slot's graph is captured at its first use; that capture's warm-up run is
+    the step itself.
+    """
+
+    def __init__(self, indexer: Indexer, B: int, n: int, *, causal: bool, max_len: int, slots: int = 2):
+        if slots < 1:
+            raise ValueError("slots must be ≥ 1")
+        dev = indexer.device
+        self.ix, self.causal, self.max_len = indexer, causal, max_len
+        self.up = torch.cuda.Stream(device=dev)
+        self.comp = torch.cuda.Stream(device=dev)
+        self.down = torch.cuda.Stream(device=dev)
+        self.slots = []
+        for _ in range(slots):
+            self.slots.append({
+                "k": torch.empty((B, n, X.DIM), dtype=torch.bfloat16, device=dev),
+                "q": torch.empty((B, n, X.HEADS, X.DIM), dtype=torch.bfloat16, device=dev),
+                "w": torch.empty((B, n, X.HEADS), dtype=torch.float32, device=dev),
+                "p": torch.empty((B,), dtype=torch.int32, device=dev),
+                "l": torch.empty((B,), dtype=torch.int32, device=dev),
+                "out": torch.empty((B, n, indexer.k), dtype=torch.int32, device=dev),
+                "graph": None,
+                "uploaded": torch.cuda.Event(),
+                "computed": torch.cuda.Event(),
+                "downloaded": torch.cuda.Event(),
+                "used": False,
+            })
+        self.count = 0
+
+    def wait(self, event: torch.cuda.Event):
+        """Make the next uploads, computes and downloads start after `event`."""
+        for st in (self.up, self.comp, self.down):
+            st.wait_event(event)
+
+    def join(self, stream=None):
+        """Make `stream` (default: the current one) wait for everything submitted."""
+        stream = stream if stream is not None else torch.cuda.current_stream(self.ix.device)
+        stream.wait_stream(self.comp)
+        stream.wait_stream(self.down)
+
+    def submit(self, h_k, h_q, h_w, h_p, h_l, h_out) -> torch.cuda.Event:
+        """One step: pinned host inputs k_new [B, n, 128] bf16, q [B, n, 64, 128]
+        bf16, w_raw [B, n, 64] fp32, positions [B], lengths [B] int32; the
+        indices land in pinned h_out [B, n, k] int32 once the returned event
+        has completed.  Refill the host inputs (or reuse h_out) only after that
+        event, or rotate several host buffers."""
+        s = self.slots[self.count % len(self.slots)]
+        self.count += 1
+        if s["used"]:
+            self.up.wait_event(s["computed"])        # the slot's inputs are free once its last step computed
+        with torch.cuda.stream(self.up):
+            for name, h in (("k", h_k), ("q", h_q), ("w", h_w), ("p", h_p), ("l", h_l)):
+                s[name].copy_(h, non_blocking=True)
+        s["uploaded"].record(self.up)
+        self.comp.wait_event(s["uploaded"])
+        if s["used"]:
+            self.comp.wait_event(s["downloaded"])    # the slot's output is free once it was read back
+        with torch.cuda.stream(self.comp):
+            if s["graph"] is None:
+                s["graph"], _ = self.ix.capture(s["k"], s["q"], s["w"], s["p"], s["l"], causal=self.causal,
+                                                max_len=self.max_len, out=s["out"])
+            else:
+                s["graph"].replay()
+        s["computed"].record(self.comp)
+        self.down.wait_event(s["computed"])
+        with torch.cuda.stream(self.down):
+            h_out.copy_(s["out"], non_blocking=True)
+        s["downloaded"].record(self.down)
+        s["used"] = True
+        return s["downloaded"]

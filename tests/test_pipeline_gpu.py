@@ -84,3 +84,55 @@ def test_e8m0_scale_storage_selects_the_same_sets(n, positions, causal):
     srt = lambda t: torch.sort(t, -1).values.cpu().numpy()
     np.testing.assert_array_equal(srt(got), srt(ref))
     np.testing.assert_array_equal(srt(out), srt(ref))
+
+
+def test_host_pipeline_matches_eager_steps_in_order():
+    """Six decode steps fed from pinned host memory through HostPipeline (copies
+    and compute overlapped, two slots) select the same sets as six eager steps,
+    and leave the same cache.  Each step's new key is built to score at the top
+    of every later step (features 1000·N(0, 1): the score grows with the key's
+    norm, positive head weights), so a step that ran before the previous
+    append landed would miss it."""
+    from sparse_attention_token_idx_b200 import binding as X
+    from sparse_attention_token_idx_b200.pipeline import HostPipeline, Indexer
+    B, steps, k = 4, 6, 64
+    base = np.array([1000, 2000, 3000, 500], np.int32)
+    case = synth.make_case("hp", 520, B, 1, base, T_cap=4096, k=k, fmt=1)
+    q = case.q
+    w_raw = np.abs(case.w_raw) + 0.5
+    rng = np.random.default_rng(521)
+    ks_new = []
+    for j in range(steps):
+        v = 1000.0 * rng.standard_normal((B, 1, 128)).astype(np.float32)
+        ks_new.append((np.ascontiguousarray(v, np.float32).view(np.uint32) >> 16).astype(np.uint16))
+    ixs = [Indexer(B, case.T_cap, case.fmt, k), Indexer(B, case.T_cap, case.fmt, k)]
+    for ix in ixs:
+        for b in range(B):
+            X.quant_append(bf16_dev(case.k_prior[b:b + 1, :base[b]]), dev(np.zeros(1, np.int32)), ix.k_cache[b:b + 1],
+                           ix.k_scale_cache[b:b + 1], case.fmt)
+    eager = []
+    for j in range(steps):
+        pos = base + j
+        out = ixs[0].step(bf16_dev(ks_new[j]), bf16_dev(q), dev(w_raw), dev(pos), dev(pos + 1), causal=False,
+                          max_len=int(pos.max()) + 1 + steps)
+        eager.append(out.cpu().numpy().copy())
+    max_len = int(base.max()) + 1 + steps
+    hp = HostPipeline(ixs[1], B, 1, causal=False, max_len=max_len)
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    h_q, h_w = pin(q.view(np.int16)).view(torch.bfloat16), pin(w_raw)
+    outs = []
+    for j in range(steps):
+        pos = base + j
+        h_out = torch.empty((B, 1, k), dtype=torch.int32).pin_memory()
+        hp.submit(pin(ks_new[j].view(np.int16)).view(torch.bfloat16), h_q, h_w, pin(pos), pin(pos + 1), h_out)
+        outs.append(h_out)
+    hp.join()
+    torch.cuda.synchronize()
+    assert X.status() == (0, 0)
+    for j in range(steps):
+        got = outs[j].numpy()
+        for b in range(B):
+            assert set(got[b, 0].tolist()) == set(eager[j][b, 0].tolist()), f"step {j} sequence {b}"
+            newer = set(range(base[b], base[b] + j))                # keys appended by the earlier steps
+            assert newer <= set(got[b, 0].tolist()), f"step {j} sequence {b} misses an earlier step's key"
+    assert torch.equal(ixs[0].k_cache, ixs[1].k_cache) and torch.equal(ixs[0].k_scale_cache, ixs[1].k_scale_cache)
