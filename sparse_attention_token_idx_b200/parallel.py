@@ -1,6 +1,12 @@
-"""Multi-GPU plumbing for the indexer: sequences are independent, so a batch
-is split into contiguous per-rank shards with no data-path collective; the
-only collectives are a barrier and the max-over-ranks reduction of timings.
+"""Multi-GPU plumbing for the indexer.
+
+* Batch sharding: sequences are independent, so a batch is split into
+  contiguous per-rank shards with no data-path collective (only a barrier and
+  the max-over-ranks reduction of timings).
+* Split-T: one sequence's keys spread over the ranks; each rank selects its
+  slice's top-k, one all-gather exchanges the (score, position) candidates and
+  every rank merges them into the sequence's top-k.
+
 Works with any torch.distributed backend (NCCL on GPUs, gloo on CPU)."""
 from __future__ import annotations
 
