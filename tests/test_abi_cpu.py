@@ -88,3 +88,26 @@ def test_product_path_fails_loudly_without_gpu():
     x = torch.zeros((4, 128), dtype=torch.bfloat16)
     with pytest.raises(binding.IdxError):
         binding.quant(x, 0)
+
+
+def test_binding_shape_checks_run_on_the_host():
+    """The Python wrappers of the widened calls reject inconsistent shapes
+    before touching the library (CPU tensors suffice)."""
+    from sparse_attention_token_idx_b200 import binding as X
+    f32, i32, bf = torch.float32, torch.int32, torch.bfloat16
+    with pytest.raises(ValueError):
+        X.gather_scores(torch.zeros((4, 16), dtype=f32), torch.zeros((3, 8), dtype=i32), 0)
+    with pytest.raises(ValueError):
+        X.merge_topk(torch.zeros((2, 4, 8), dtype=i32), 8)                       # not [G, rows, kin, 2]
+    with pytest.raises(ValueError):
+        X.sparse_mla_decode(torch.zeros((2, 16, 512), dtype=bf), torch.zeros((2, 64, 576), dtype=bf),
+                            torch.zeros((2, 8), dtype=i32), 0.1)                # 512 query features
+    with pytest.raises(ValueError):
+        X.sparse_mla_decode(torch.zeros((2, 16, 576), dtype=bf), torch.zeros((3, 64, 576), dtype=bf),
+                            torch.zeros((2, 8), dtype=i32), 0.1)                # batch mismatch
+    with pytest.raises(ValueError):
+        X.front_quant_append(torch.zeros((2, 1, 64, 128), dtype=bf), torch.zeros((2, 1, 64), dtype=f32),
+                             torch.zeros((2, 1, 128), dtype=bf), torch.zeros((2, 1, 16), dtype=f32),
+                             torch.zeros((2, 1, 32), dtype=f32), torch.ones(128), torch.zeros(128), 1e-6,
+                             torch.zeros(2, dtype=i32), torch.zeros((2, 64, 128), dtype=torch.uint8),
+                             torch.zeros((2, 64), dtype=f32), 0)               # cos table of 16, not 32
