@@ -49,6 +49,9 @@ def weak_scaling_total(per_rank_units: float) -> float:
 # its own slice's k best), which the broadcast-and-compare of the reference
 # forward only asserts across ranks.
 
+_NEG_INF_BITS = -8388608   # 0xFF800000, the float32 bits of −inf, as int32
+
+
 def key_slice(T_cap: int, rank: int, world: int, align: int = 128) -> tuple[int, int]:
     """Cache positions [lo, hi) that `rank` holds: contiguous slices of a
     multiple of `align` positions (the last may be shorter or empty)."""
@@ -89,10 +92,14 @@ def slice_candidates(q_fp8, w, k_cache, k_scale_cache, lengths, lo: int, hi: int
     int32 [B, k, 2] (score bits, global position; −1 empty).  lengths [B] int32
     are the whole sequences' lengths."""
     from . import binding as X
+    B = q_fp8.shape[0]
+    span = hi - lo
+    if span <= 0:                        # this rank holds no positions: only empty candidates (−inf, −1)
+        cand = torch.full((B, k, 2), -1, dtype=torch.int32, device=q_fp8.device)
+        cand[..., 0] = _NEG_INF_BITS
+        return cand
     counts = slice_counts(lengths, lo, hi)
     eff = counts.clamp(min=1)            # an empty slice is scored as one key and dropped by the gather
-    span = hi - lo
-    B = q_fp8.shape[0]
     scores = X.score_visible(q_fp8, w, k_cache, k_scale_cache, eff, False, span, stream=stream)
     idx_local = X.topk(scores, eff, False, k, span, stream=stream)
     return X.gather_scores(scores.reshape(B, span), idx_local.reshape(B, k), lo, counts=counts, stream=stream)

@@ -253,3 +253,17 @@ def test_two_gloo_ranks_split_t_decode_orchestration():
         assert p.exitcode == 0
     assert all(all(r[1]) for r in res), "split-T result differs from the whole-sequence top-k"
     assert all(r[2] == 3 * 40 for r in res)
+
+
+def test_empty_key_slice_contributes_only_empty_candidates():
+    """A rank whose slice holds no positions (more ranks than 128-position
+    blocks) returns (−inf, −1) pairs without calling the library."""
+    import torch
+    from sparse_attention_token_idx_b200.parallel import slice_candidates
+    lo, hi = key_slice(256, 3, 4)
+    assert lo == hi == 256
+    c = slice_candidates(torch.zeros((2, 1, 64, 128), dtype=torch.uint8), torch.zeros((2, 1, 64)),
+                         torch.zeros((2, 0, 128), dtype=torch.uint8), torch.zeros((2, 0)),
+                         torch.tensor([200, 256], dtype=torch.int32), lo, hi, 16)
+    assert c.shape == (2, 16, 2) and torch.all(c[..., 1] == -1)
+    assert torch.all(torch.isneginf(c[..., 0].contiguous().view(torch.float32)))
