@@ -37,7 +37,7 @@ What it computes, step by step, with the passage each step follows:
 * ``MASK_BOUND_BF16``, ``scores_bf16`` — the NKI page's Notes: masked slots
   hold a finite bound instead of −inf for consumers that read bfloat16.
 
-Readings taken where the pages are silent (each one also listed in the design doc):
+Readings taken where the pages are silent:
 
 * H_128 is the Sylvester matrix in natural order, H[i, j] = (−1)^popcount(i & j).
 * The rotation runs on the bf16 inputs in float64 as a butterfly with strides

@@ -18,7 +18,7 @@ parts gives the same product as adding their two scores, as the page says).
                                                           before the value
                                                           up-projection)
 
-Readings (also listed in the design doc):
+Readings taken where the pages are silent:
 * queries and the cache are bf16 values; everything here is float64;
 * a selection entry of −1 (the indexer's padding) selects nothing; a row with
   no selected position has output 0;
