@@ -7,12 +7,20 @@
  *   scores:  S[t,s] = k_scale[s] · Σ_{h<64} w[t,h] · ReLU(q_fp8[t,h] · k_fp8[s]);
  *   select:  the min(k, visible) highest-scoring cached positions per query row.
  *
+ * Around that path: the front end before it (query RoPE, key LayerNorm + RoPE,
+ * fused with the quantiser: idx_front_quant_append), the attention after it
+ * (sparse latent attention over the selected positions: idx_sparse_mla_decode),
+ * and split-T selection of one sequence over several GPUs (idx_gather_scores,
+ * idx_merge_topk).
+ *
  * Sources (web pages on DeepSeek-V3.2-Exp's lightning indexer):
  *   "Index scores"          — score equation S^I, fp8_index docstring, Indexer.forward excerpt;
  *   "Index key cache"       — k_cache / k_scale_cache buffers, append before scoring;
  *   "Hadamard rotation"     — rotation equation and orthonormality note;
  *   NKI "DeepSeek-V3.2 Sparse Indexer Kernel API Reference" — caller-owned cache written in
- *                             place, int32 positions, int32 unordered top-k set.
+ *                             place, int32 positions, int32 unordered top-k set, finite mask
+ *                             bound, front-end parameters (cos / sin tables, LayerNorm gain, bias);
+ *   "Join query parts"      — MQA decode excerpt: the attention that consumes the selection.
  *
  * Conventions for every call below.
  *   - All array arguments are DEVICE pointers to row-major, contiguous memory
