@@ -210,6 +210,60 @@ def test_rotate_equals_exact_signed_sums_then_two_roundings():
             assert Fraction(float(got[r, i])) == want
 
 
+def _bf16_rne_bits(p: np.ndarray) -> np.ndarray:
+    """Round-to-nearest-even of float64 values onto bf16 (normal range only),
+    done on the IEEE-754 bit pattern: keep the sign, exponent and top 7
+    fraction bits, round on the 45 dropped bits (ties to an even kept field)."""
+    u = np.ascontiguousarray(p, np.float64).view(np.uint64)
+    drop = np.uint64(45)
+    half = np.uint64(1) << np.uint64(44)
+    odd = (u >> drop) & np.uint64(1)
+    r = (u + (half - np.uint64(1)) + odd) & ~((np.uint64(1) << drop) - np.uint64(1))
+    return r.view(np.float64)
+
+
+def test_rotate_rounds_once_from_float64_on_many_rows():
+    """The rotation's reading is one float64 multiply of the exact butterfly sum,
+    then ONE round-to-nearest-even to bf16.  A plausible slip is an fp32
+    intermediate (round to fp32, then to bf16): it differs only where the fp32
+    value lands exactly on a bf16 midpoint, about one row in a thousand.  This
+    pin checks 2·10^5 rows of the workloads' distribution against sums taken
+    independently of the butterfly (scipy's Hadamard matrix as a BLAS product,
+    exact because every partial sum is a multiple of the row's smallest bf16
+    quantum below 2^53) and a bit-level rounding, and requires that the rows
+    hold enough double-rounding witnesses for the slip to fail it."""
+    rng = np.random.default_rng(31)
+    rows = 200_000
+    raw = rng.standard_normal((rows, 128)).astype(np.float32)
+    ch = rng.choice(128, size=2, replace=False)
+    raw[:, ch] *= 20
+    bits = synth._to_bf16_bits(raw)
+    x = O.bf16_bits_to_f64(bits)
+    # exactness of the float64 sums: exponent span of each row's nonzero values
+    _, e = np.frexp(np.where(x == 0, 1.0, np.abs(x)))
+    span = np.where(x == 0, e.min(), e).max(-1) - np.where(x == 0, e.max(), e).min(-1)
+    assert span.max() <= 38
+    y = x @ scipy.linalg.hadamard(128).astype(np.float64).T
+    p = y * O.INV_SQRT_D_F64                       # one IEEE float64 multiply
+    want = _bf16_rne_bits(p)
+    got = O.bf16_bits_to_f64(O.rotate(bits))
+    np.testing.assert_array_equal(got, want)
+    # the same check on the fp32 route would fail here: count its witnesses
+    f32 = p.astype(np.float32).astype(np.float64)
+    double = _bf16_rne_bits(f32)
+    witness_rows = np.unique(np.nonzero(double != want)[0])
+    assert witness_rows.size >= 50, witness_rows.size
+    # and those rows again in exact rationals (Fraction sums, exact rounding)
+    Hs = scipy.linalg.hadamard(128)
+    c = Fraction(O.INV_SQRT_D_F64)
+    for r in witness_rows[:8]:
+        cols = np.nonzero(double[r] != want[r])[0]
+        xs = [Fraction(float(v)) for v in x[r]]
+        for i in cols:
+            ysum = sum(xs[j] if Hs[i, j] > 0 else -xs[j] for j in range(128))
+            assert Fraction(float(got[r, i])) == bf16_exact(Fraction(float(ysum * c)))
+
+
 # --------------------------------------------------------------------------- quant
 def _rows(seed, n=200):
     rng = np.random.default_rng(seed)
@@ -447,6 +501,24 @@ def test_folded_weights_reproduce_the_unfolded_score_equation():
                 page = (1.0 / (math.sqrt(64) * math.sqrt(128))) * (
                     case.w_raw[b, i].astype(np.float64)[:, None] * np.maximum(qbar @ kbar[:vis].T, 0)).sum(0)
                 assert np.all(np.abs(S[b, i, :vis] - page) <= 4e-7 * E[b, i, :vis] + 1e-30)
+
+
+def test_folded_weights_equal_the_page_expression_in_torch_fp32():
+    """Bit for bit against the Indexer.forward excerpt ("Index scores" page,
+    the two weight lines) evaluated by torch on the CPU in fp32: the weight
+    projection times 64^-0.5, then times the query scale, then times the
+    softmax scale 128^-0.5, each product rounded to fp32.  A reordered fold
+    or a constant one ulp off fails here."""
+    rng = np.random.default_rng(77)
+    w_raw = rng.standard_normal((512, 64)).astype(np.float32)
+    q_bits = synth._to_bf16_bits(rng.standard_normal((512, 64, 128)).astype(np.float32) *
+                                 np.exp(rng.uniform(-6, 6, (512, 64, 1))).astype(np.float32))
+    for fmt in (0, 1):
+        _, q_scale, w = O.quant_queries(q_bits, w_raw, fmt)
+        n_heads, head_dim = 64, 128
+        wt = torch.from_numpy(w_raw) * n_heads ** -0.5
+        wt = wt.unsqueeze(-1) * torch.from_numpy(q_scale).unsqueeze(-1) * head_dim ** -0.5
+        np.testing.assert_array_equal(w.view(np.uint32), wt.squeeze(-1).numpy().view(np.uint32))
 
 
 def test_append_writes_exactly_the_requested_slots():
