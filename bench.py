@@ -1,15 +1,18 @@
 """Benchmark of the lightning-indexer hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl ours|reference]
+                    [--no-prefill] [--no-cpu-baseline]
 
 A step is one whole indexer call on one batch: append the new keys to the FP8
 cache (rotate + quantise + store), quantise the queries and fold the head
-weights, then the fused score + top-k over every cached key.  The default
+weights, then score + top-k over every visible cached key.  The headline
 workload is the bandwidth-bound decode case (B = 128 sequences, 16 384 cached
 keys each, ue8m0 scales, k = 2048): its 277 MB FP8 cache is larger than the
-126 MB L2, so consecutive steps stream it from HBM.  Other workloads
-(--workload 0…4) are for measurement notes; the prefill ones report FP8
-TFLOP/s.
+126 MB L2, so consecutive steps stream it from HBM.  The same run then times
+the two prefill workloads (4096 causal rows from position 0; 2 × 2048 rows
+appended at 14 336) and reports them under "prefill" with their FP8 TFLOP/s
+against the tensor peak; their steps are timed one by one with an L2 flush
+between them.  --workload 0…4 times one workload alone.
 
 Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
 sequences (weak scaling, no data-path collective); times are the max over
@@ -37,6 +40,9 @@ DEFAULT_WORKLOAD = 2
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP8_PER_BF16 = 2.0            # nominal dense fp8 : bf16 tensor ratio on B200
+DATASHEET_FP8_TFLOPS = 4500.0  # B200 dense FP8, datasheet (context beside the measured-derived peak)
+NOMINAL_HBM_GBS = 8000.0      # HBM3e nominal figure the decode target is also quoted against
+PREFILL_WORKLOADS = (3, 4)
 KEY_BYTES = 128 + 4           # one cached key: 128 e4m3 codes + fp32 scale
 ROW_BYTES_IN = 64 * 128 + 64 * 4   # one query row: 64 heads of e4m3 codes + 64 fp32 weights
 PROFILE_SCORE = os.path.join(ROOT, "profiles", "score_topk_decode_b128_t16384.md")
@@ -149,7 +155,18 @@ def workload_numbers(case):
     return keys, flops, key_rows, score_bytes
 
 
-def run_ours(args, rank, world, local_rank):
+def l2_flush_buffer(torch, dev):
+    """A buffer twice the L2 size; writing it evicts the previous step's lines."""
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size or (126 << 20)
+    return torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+
+def measure(args, widx, dev, world, headline):
+    """One workload on this rank's GPU: fill the cache, capture the step in a
+    CUDA graph, warm up, then time K whole steps, the dominant kernel(s) on
+    their own, and K end-to-end steps from pinned host memory.  Decode steps
+    stream a cache larger than L2 back to back; prefill steps are timed one
+    by one with an L2 flush between them (not timed)."""
     import torch
     import torch.distributed as dist
 
@@ -158,14 +175,12 @@ def run_ours(args, rank, world, local_rank):
     from sparse_attention_token_idx_b200.parallel import max_over_ranks
     from sparse_attention_token_idx_b200.pipeline import HostPipeline, Indexer
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    case = synth.workload(args.workload)
+    case = synth.workload(widx)
     B, n = case.B, case.n
     bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
     dv = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
 
-    e8m0 = getattr(args, "scale_storage", "f32") == "e8m0"
+    e8m0 = headline and getattr(args, "scale_storage", "f32") == "e8m0"
     if e8m0 and (case.fmt != 1 or case.n > 2):
         raise SystemExit("--scale-storage e8m0 applies to the ue8m0 decode workload (2)")
     ix = Indexer(B, case.T_cap, case.fmt, case.k, device=dev, scale_storage="e8m0" if e8m0 else "f32")
@@ -190,9 +205,9 @@ def run_ours(args, rank, world, local_rank):
     if e8m0:   # one scale byte per cached key instead of four
         score_bytes -= 3 * key_rows
 
-    # the kernel the roofline is about, timed on its own stream with events: the
-    # tcgen05 scorer writing the workspace when the step uses one (the step's
-    # dominant kernel; its top-k timed apart), else the fused score + top-k
+    # the kernel the roofline is about: the tcgen05 scorer writing the
+    # workspace when the step uses one (its top-k timed apart), else the fused
+    # score + top-k
     ws_bytes = X.workspace_size(B, n, max_len, case.k)
     if ws_bytes:   # the scorer writes fp32 score rows instead of indices
         score_bytes += B * n * (4 * max_len - 4 * case.k)
@@ -210,9 +225,7 @@ def run_ours(args, rank, world, local_rank):
         X.topk(sc_view, lengths, case.causal, case.k, max_len, out=out)
 
     graph, g_out = ix.capture(k_new, q, w_raw, positions, lengths, causal=case.causal, max_len=max_len)
-
-    def step():
-        graph.replay()
+    flush = None if key_rows * KEY_BYTES > 2 * 126e6 else l2_flush_buffer(torch, dev)
 
     if e8m0:
         X.quant_queries(q, w_raw, case.fmt, q_fp8, w)
@@ -220,47 +233,46 @@ def run_ours(args, rank, world, local_rank):
     else:
         X.quant_queries_append(q, w_raw, k_new, positions, ix.k_cache, ix.k_scale_cache, case.fmt, q_fp8, w)
     for _ in range(args.warmup):
-        step()
+        graph.replay()
         score_only()
     torch.cuda.synchronize()
     code, bits = X.status()
     if code != 0:
         raise RuntimeError(f"device error during warm-up: status {code}, bits {bits}")
 
+    def back_to_back(fn, count):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(count):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
     # -------------------------------------------------------------- timed region: whole steps
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(torch.cuda.current_device())
     with sampler:
-        t0.record(stream)
-        for i in range(args.steps):
-            step()
-        t1.record(stream)
-        torch.cuda.synchronize()
+        if flush is None:
+            ms = back_to_back(graph.replay, args.steps)
+        else:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for a, b in evs:
+                flush.zero_()
+                a.record(stream)
+                graph.replay()
+                b.record(stream)
+            torch.cuda.synchronize()
+            ms = sum(a.elapsed_time(b) for a, b in evs)
     if world > 1:
         dist.barrier()
-    ms = t0.elapsed_time(t1)
-    # the fused score + top-k kernel alone, launch by launch on the same stream
-    n_k = min(args.steps, 500)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_k)]
-    for i in range(n_k):
-        evs[i][0].record(stream)
-        score_only()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    score_ms = sum(a.elapsed_time(b) for a, b in evs) / n_k
-    topk_ms = None
-    if ws_bytes:
-        n_t = min(args.steps, 50)
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        for _ in range(n_t):
-            topk_only()
-        s1.record(stream)
-        torch.cuda.synchronize()
-        topk_ms = s0.elapsed_time(s1) / n_t
+    # the dominant kernel alone: back-to-back launches between two events
+    n_k = max(3, min(args.steps, 200))
+    score_ms = back_to_back(score_only, n_k) / n_k
+    topk_ms = back_to_back(topk_only, n_k) / n_k if ws_bytes else None
     code, bits = X.status()
     if code != 0:
         raise RuntimeError(f"device error in the timed region: status {code}, bits {bits}")
@@ -305,10 +317,12 @@ def run_ours(args, rank, world, local_rank):
     if topk_ms is not None:
         topk_ms = max_over_ranks([topk_ms], device=dev)[0]
     topk_bytes = B * n * 4 * (max_len + case.k) if ws_bytes else None   # score rows read, indices written
+    launches_per_step = (3 if (ws_bytes or e8m0) else 2)
+    del graph, hp, ix, ws
     return dict(case=case, e8m0=e8m0, keys=keys, flops=flops, key_rows=key_rows, score_bytes=score_bytes, ms=ms,
                 score_ms=score_ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
-                clocks=sampler.summary(), launches=(3 if (ws_bytes or e8m0) else 2) * args.steps, topk_ms=topk_ms,
-                topk_bytes=topk_bytes, two_pass=bool(ws_bytes))
+                clocks=sampler.summary(), launches=launches_per_step * args.steps, topk_ms=topk_ms,
+                topk_bytes=topk_bytes, two_pass=bool(ws_bytes), l2_flushed=flush is not None)
 
 
 def case_pinned(torch, a):
@@ -411,6 +425,9 @@ def main():
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="time only the selected workload (by default the decode headline also runs "
+                         "the two prefill workloads and reports them under 'prefill')")
     ap.add_argument("--scale-storage", choices=["f32", "e8m0"], default="f32",
                     help="key scales as float32 (the workloads' layout) or one e8m0 byte per key "
                          "(ue8m0 workloads only)")
@@ -436,15 +453,36 @@ def main():
 
     import torch
     import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
     if world > 1:
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
-    try:
-        r = run_ours(args, rank, world, local_rank)
-    finally:
-        pass
-    case = r["case"]
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     hbm, bf16, bf16_sus, peak_src = measured_peaks()
+    r = measure(args, args.workload, dev, world, headline=True)
+    line = result_line(r, args, world, hbm, bf16, peak_src)
+    if args.workload == DEFAULT_WORKLOAD and not args.no_prefill:
+        # the prefill half of the metric: FP8 TFLOP/s of the two prefill workloads
+        line["prefill"] = {}
+        for widx in PREFILL_WORKLOADS:
+            rp = measure(args, widx, dev, world, headline=False)
+            sub = result_line(rp, args, world, hbm, bf16, peak_src)
+            for key in ("metric", "n_gpus", "steps", "warmup", "higher_is_better", "scaling", "vs_baseline",
+                        "data"):
+                sub.pop(key, None)
+            line["prefill"][str(widx)] = sub
+        line["gpu_launches"] += sum(p["gpu_launches"] for p in line["prefill"].values())
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(r["case"])
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def result_line(r, args, world, hbm, bf16, peak_src):
+    case = r["case"]
     step_s = r["ms"] / 1e3 / args.steps
     value = r["keys"] * world / step_s
     e2e_value = r["keys"] * world / (r["e2e_ms"] / 1e3 / r["e2e_steps"])
@@ -454,17 +492,27 @@ def main():
         peak = bf16 * FP8_PER_BF16
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "traffic": None, "peak_source": f"{peak_src} bf16 burst x nominal fp8/bf16 ratio {FP8_PER_BF16}",
-                "kernel": "score (tcgen05 FP8 scorer, fp32 scores to the workspace)",
-                "kernel_us": r["score_ms"] * 1e3, "algorithmic_flops": r["flops"]}
+                "frac_of_datasheet_fp8": achieved / DATASHEET_FP8_TFLOPS,
+                "kernel": "flat_score_kernel (tcgen05 FP8 scorer, fp32 scores to the workspace)",
+                "kernel_us": r["score_ms"] * 1e3, "algorithmic_flops": r["flops"],
+                "timing": "back-to-back launches between two CUDA events"}
     else:
         achieved = r["score_bytes"] / score_s / 1e9
         traffic = (profile_traffic(PROFILE_SCORE, r["key_rows"])
                    if args.workload == DEFAULT_WORKLOAD and not r["e8m0"] else None)
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": traffic, "peak_source": f"{peak_src} copy bandwidth",
-                "kernel": "score (tcgen05 FP8 scorer, fp32 scores to the workspace)" if r["two_pass"]
-                else "score_topk (fused)",
-                "kernel_us": r["score_ms"] * 1e3, "algorithmic_bytes": r["score_bytes"]}
+                "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                "target_basis": "the 70% decode target is read against the measured copy peak (frac); "
+                                "frac_of_nominal_8tbs is the same time against 8 TB/s",
+                "kernel": "flat_score_kernel (tcgen05 FP8 scorer, fp32 scores to the workspace)" if r["two_pass"]
+                else "score_kernel (fused score + top-k)",
+                "kernel_us": r["score_ms"] * 1e3, "algorithmic_bytes": r["score_bytes"],
+                "timing": "back-to-back launches between two CUDA events"}
+    l2 = ("L2 flushed (a write of twice the L2 size) before each step, outside the timed events"
+          if r["l2_flushed"] else
+          "inputs larger than L2: %.0f MB FP8 cache streamed per step"
+          % (r["key_rows"] * (KEY_BYTES - 3 * r["e8m0"]) / 1e6))
     line = {
         "metric": metric_name(case), "value": value, "unit": "keys/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -472,10 +520,7 @@ def main():
         "config": {"workload": case.name + (", e8m0 scale bytes" if r["e8m0"] else ""), "B": case.B, "n": case.n,
                    "T_cap": case.T_cap, "k": case.k,
                    "scale_storage": "e8m0 bytes (129 B/key)" if r["e8m0"] else "fp32 (132 B/key)",
-                   "heads": 64, "head_dim": 128, "fmt": ["fp32", "ue8m0"][case.fmt],
-                   "l2": ("inputs larger than L2: %.0f MB FP8 cache streamed per step"
-                          % (r["key_rows"] * (KEY_BYTES - 3 * r["e8m0"]) / 1e6))
-                   if r["key_rows"] * KEY_BYTES > 126e6 else "L2-resident working set (not flushed)",
+                   "heads": 64, "head_dim": 128, "fmt": ["fp32", "ue8m0"][case.fmt], "l2": l2,
                    "parallelism": f"dp{world} (independent sequences per rank)"},
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": "keys/s", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
@@ -485,17 +530,13 @@ def main():
     }
     if case.causal:
         line["tflops"] = r["flops"] * world / step_s / 1e12      # whole step (quantise + score + top-k)
+        line["e2e"]["tflops"] = r["flops"] * world / (r["e2e_ms"] / 1e3 / r["e2e_steps"]) / 1e12
     if r["topk_ms"] is not None:
-        line["topk_us"] = r["topk_ms"] * 1e3
-        line["topk"] = {"us": r["topk_ms"] * 1e3, "algorithmic_bytes": r["topk_bytes"],
-                        "achieved_gbs": r["topk_bytes"] / (r["topk_ms"] / 1e3) / 1e9}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(case)
-    if rank == 0:
-        print(json.dumps(line))
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+        line["topk"] = {"kernel": "topk_row_kernel", "us": r["topk_ms"] * 1e3,
+                        "algorithmic_bytes": r["topk_bytes"],
+                        "achieved_gbs": r["topk_bytes"] / (r["topk_ms"] / 1e3) / 1e9,
+                        "frac_of_measured_hbm": r["topk_bytes"] / (r["topk_ms"] / 1e3) / 1e9 / hbm}
+    return line
 
 
 def metric_name(case):

@@ -347,9 +347,11 @@ IDX_API int idx_score_topk_ex(const uint8_t* q_fp8, const float* w, const uint8_
  * Prefill-shaped calls keep their score workspace in a buffer the library
  * owns: a file-scope device array of 64 MiB (B·n·max_len ≤ 16 Mi scores),
  * held on every GPU that loads the library until the process exits.  Larger
- * calls return IDX_ERR_SCRATCH; decode-shaped calls need no scratch.
- *   - The first call on a device looks up the buffer's device address (no
- *     allocation); make that first call before any stream capture.
+ * calls return IDX_ERR_SCRATCH before anything is enqueued — for example two
+ * sequences of 2048 new rows over 16 384 keys (256 MiB of scores): call
+ * idx_score_topk with a workspace for those.  Decode-shaped calls need no scratch.
+ *   - The first call on a device, of any shape, looks up the buffer's device
+ *     address (no allocation); make that first call before any stream capture.
  *   - Every call reuses the same buffer and rewrites all of the part it uses,
  *     so nothing needs clearing, but calls that overlap on the GPU (other
  *     streams, other threads) race on it: serialise them.

@@ -24,7 +24,8 @@ What it computes, step by step, with the passage each step follows:
 * ``index_scores``     — "Index scores" page, score equation S^I and the
   ``fp8_index`` docstring (FP8 logits → ReLU → × weight → sum over heads →
   × key scale), plus the causal mask added in prefill (``Indexer.forward``
-  excerpt).
+  excerpt).  ``index_scores_rows`` computes the same for many rows of one
+  sequence with matrix products as its steps (full-size checks).
 * ``topk``             — ``Indexer.forward`` excerpt (top min(index_topk, ·)
   positions per row) and the NKI "DeepSeek-V3.2 Sparse Indexer Kernel API
   Reference" page, Notes and return types (int32, an unordered set).
@@ -340,6 +341,39 @@ def index_scores(q_codes, w, k_cache, k_scale_cache, lengths, causal, ncols=None
             S[b, i, :v] = ks[:v] * np.sum(wi * np.maximum(logits, 0.0), axis=0)
             if with_bound:
                 E[b, i, :v] = np.abs(ks[:v]) * np.sum(np.abs(wi * logits), axis=0)
+    return S, E
+
+
+def index_scores_rows(q_codes, w, k_codes, k_scale, vis):
+    """S and E of several query rows of one sequence, as ``index_scores``
+    defines them, with library matrix products as the steps: the logits of all
+    rows against the first max(vis) keys as one product (exact: every FP8
+    product and partial sum is a multiple of 2^-18 below 2^53), then the
+    head-weighted ReLU sum and the bound as batched products over the heads
+    (float64; only the summation order over the 64 heads differs from
+    ``index_scores``).
+
+    q_codes [R, 64, 128] uint8; w [R, 64] float32; k_codes [>= max(vis), 128]
+    uint8 and k_scale [>= max(vis)] float32 of the sequence; vis [R] visible key
+    counts.  Returns S, E [R, max(vis)] float64, −inf / 0 from each row's
+    visible count on."""
+    vis = np.asarray(vis, np.int64)
+    R, V = len(vis), int(vis.max()) if len(vis) else 0
+    S = np.full((R, V), -np.inf)
+    E = np.zeros((R, V))
+    if V == 0:
+        return S, E
+    kd = e4m3_decode(k_codes[:V])                                   # [V, 128]
+    ks = np.asarray(k_scale[:V], np.float64)
+    qd = e4m3_decode(np.asarray(q_codes, np.uint8)).reshape(R * H, D)
+    logits = (qd @ kd.T).reshape(R, H, V)                           # exact
+    wi = np.asarray(w, np.float64)[:, None, :]                      # [R, 1, 64]
+    S[:] = (wi @ np.maximum(logits, 0.0))[:, 0, :] * ks
+    E[:] = (np.abs(wi) @ np.abs(logits))[:, 0, :] * np.abs(ks)
+    cols = np.arange(V)[None, :]
+    past = cols >= vis[:, None]
+    S[past] = -np.inf
+    E[past] = 0.0
     return S, E
 
 

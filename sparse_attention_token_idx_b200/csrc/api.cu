@@ -6,7 +6,9 @@
 
 #include <atomic>
 #include <cstdint>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "api_internal.h"
 #include "ptx.cuh"
@@ -88,6 +90,20 @@ int smem_per_sm() {
     cache[d].store(v);
   }
   return v;
+}
+
+int ensure_smem_limit(const void* func, int smem) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, int> limits;   // (device, kernel) → bytes set
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return check_launch();
+  std::lock_guard<std::mutex> lock(mu);
+  int& have = limits[{dev, func}];
+  if (have >= smem) return IDX_OK;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return check_launch();
+  have = smem;
+  return IDX_OK;
 }
 
 int check_launch() {

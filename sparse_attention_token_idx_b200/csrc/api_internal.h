@@ -12,6 +12,10 @@ int num_sms();                       // SM count of the current device (cached p
 int check_launch();                  // IDX_OK, or IDX_ERR_LAUNCH after recording cudaGetLastError()
 int max_dynamic_smem();              // opt-in shared memory per block of the current device
 int smem_per_sm();                   // shared memory per SM of the current device
+// Raise `func`'s dynamic shared-memory limit to at least `smem` bytes on the
+// current device (remembered per device and kernel, so that a process driving
+// several GPUs sets it once on each).  IDX_OK, or check_launch()'s code.
+int ensure_smem_limit(const void* func, int smem);
 
 // Tensor map for a [outer, mid, inner] uint8 array (row pitch `inner` bytes,
 // plane pitch mid·inner bytes), box {128 bytes, box_rows, 1}, 128-byte swizzle.

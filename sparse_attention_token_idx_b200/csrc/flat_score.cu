@@ -453,12 +453,7 @@ int launch_flat_t(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, 
   if (!make_tmap_scales(&ts, k_scale_cache, scale_fmt, static_cast<uint64_t>(T_cap), static_cast<uint64_t>(B), kFKeys))
     return IDX_ERR_ALIGN;
   auto kern = flat_score_kernel<NT, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>;
-  static int configured_smem = -1;   // per instantiation
-  if (configured_smem < smem) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return check_launch();
-    configured_smem = smem;
-  }
+  if (const int r = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem)) return r;
   FlatParams p;
   p.w = w;
   p.lengths = lengths;

@@ -146,13 +146,7 @@ extern "C" int idx_sparse_mla_decode(const uint16_t* q, const uint16_t* kv, cons
   const int64_t blocks = static_cast<int64_t>(B) * (H / kMlaHeads);
   if (blocks > 0x7FFFFFFF) return IDX_ERR_SHAPE;
   const int smem = static_cast<int>(sizeof(MlaSmem));
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(sparse_mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return check_launch();
-    configured = true;
-  }
+  if (const int r = ensure_smem_limit(reinterpret_cast<const void*>(sparse_mla_decode_kernel), smem)) return r;
   sparse_mla_decode_kernel<<<static_cast<unsigned>(blocks), kMlaThreads, static_cast<size_t>(smem),
                              reinterpret_cast<cudaStream_t>(stream)>>>(q, kv, indices, H, T_cap, k, softmax_scale,
                                                                        out);

@@ -23,6 +23,8 @@
 #include <cuda_runtime.h>
 #include <atomic>
 #include <cstdint>
+#include <map>
+#include <mutex>
 
 #include "api_internal.h"
 #include "ptx.cuh"
@@ -531,12 +533,7 @@ int launch_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, c
     return IDX_ERR_ALIGN;
 
   auto kern = score_kernel<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>;
-  static int configured_smem = -1;   // per instantiation
-  if (configured_smem < smem) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return check_launch();
-    configured_smem = smem;
-  }
+  if (const int r = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem)) return r;
   ScoreParams p;
   p.w = w;
   p.k_scale = k_scale_cache;
@@ -727,19 +724,26 @@ namespace {
 constexpr size_t kStaticScratchBytes = size_t(64) << 20;   // 64 MiB: B·n·max_len ≤ 16 Mi scores
 static __device__ __align__(256) float g_static_scratch[kStaticScratchBytes / sizeof(float)];
 
-std::atomic<float*> g_static_scratch_addr[64];
-
 // Device address of g_static_scratch on the current device (host code cannot
-// use the symbol itself: on the host it only names a stand-in).
+// use the symbol itself: on the host it only names a stand-in), looked up once
+// per device.  nullptr when the lookup fails (its CUDA error is recorded).
 float* static_scratch() {
+  static std::mutex mu;
+  static std::map<int, float*> addr;   // device ordinal → address
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  float* a = g_static_scratch_addr[dev].load();
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    check_launch();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  float*& a = addr[dev];
   if (!a) {
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) {
+      check_launch();
+      return nullptr;
+    }
     a = static_cast<float*>(ptr);
-    g_static_scratch_addr[dev].store(a);
   }
   return a;
 }
@@ -756,14 +760,13 @@ extern "C" int idx_score_topk_noalloc(const uint8_t* q_fp8, const float* w, cons
   if (!indices) return IDX_ERR_NULL;
   const size_t need = idx_workspace_size(B, n, max_len, k);
   if (need > kStaticScratchBytes) return IDX_ERR_SCRATCH;
+  // the buffer's address is looked up on the first call on a device, whatever
+  // the call's shape, so that a decode-shaped first call also does the lookup
+  float* scratch = static_scratch();
+  if (!scratch) return IDX_ERR_LAUNCH;
   if (need == 0)   // decode-shaped: the single kernel needs no scratch
     return idx_score_topk(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal, k, indices,
                           nullptr, 0, stream);
-  float* scratch = static_scratch();
-  if (!scratch) {
-    check_launch();   // records the CUDA error of the failed lookup
-    return IDX_ERR_LAUNCH;
-  }
   return idx_score_topk(q_fp8, w, k_cache, k_scale_cache, lengths, B, n, T_cap, max_len, causal, k, indices,
                         scratch, kStaticScratchBytes, stream);
 }

@@ -482,12 +482,7 @@ extern "C" int idx_topk(const float* scores, const int32_t* lengths, int B, int 
     const RowLayout L = row_layout(chunk_cap, list_cap, cand_cap);
     const int smem = L.total + 128;
     if (smem > max_dynamic_smem()) return IDX_ERR_SHAPE;
-    static int configured_row = -1;
-    if (configured_row < smem) {
-      if (cudaFuncSetAttribute(topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return check_launch();
-      configured_row = smem;
-    }
+    if (const int r = ensure_smem_limit(reinterpret_cast<const void*>(topk_row_kernel), smem)) return r;
     const DebugState dbg = debug_state();
     RowParams rp{scores, lengths, indices, ld, B, n, max_len, causal, k, chunk_cap, list_cap, cand_cap,
                  dbg.budget_ns, device_error_word(), (dbg.flags & 2u) ? trace_buffer() : nullptr};
@@ -508,12 +503,7 @@ extern "C" int idx_topk(const float* scores, const int32_t* lengths, int B, int 
   const int smem = 128 + static_cast<int>(sizeof(SelectSmem)) + (kHistBins + cand_cap) * 4 + chunk_cap * 4;
   if (smem > max_dynamic_smem()) return IDX_ERR_SHAPE;
   if (rows * G > 0x7FFFFFFF) return IDX_ERR_SHAPE;
-  static int configured = -1;
-  if (configured < smem) {
-    if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return check_launch();
-    configured = smem;
-  }
+  if (const int r = ensure_smem_limit(reinterpret_cast<const void*>(topk_kernel), smem)) return r;
   TopkParams p{scores, lengths, indices, ld, B, n, max_len, causal, k, G, chunk_cap, cand_cap, device_error_word(),
                (debug_state().flags & 2u) ? trace_buffer() : nullptr};
   if (!p.err) return check_launch();
@@ -558,12 +548,7 @@ extern "C" int idx_merge_topk(const idx_cand_t* cand, int G, int64_t rows, int k
   const int smem = merge_layout(m4, cand_cap).total + 128;
   const bool pairs2 = (kin % 2) == 0 && (reinterpret_cast<uintptr_t>(cand) & 15u) == 0;
   auto kern = pairs2 ? merge_topk_kernel<true> : merge_topk_kernel<false>;
-  static int configured[2] = {-1, -1};
-  if (configured[pairs2] < smem) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return check_launch();
-    configured[pairs2] = smem;
-  }
+  if (const int r = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem)) return r;
   kern<<<static_cast<unsigned>(rows), kMergeThreads, static_cast<size_t>(smem),
          reinterpret_cast<cudaStream_t>(stream)>>>(cand, G, rows, kin, k, cand_cap, out);
   return check_launch();

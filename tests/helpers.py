@@ -127,3 +127,53 @@ def check_topk_exact_row(got_row: np.ndarray, scores: np.ndarray, vis: int, k: i
     assert np.all(sel[s > tau]), "an element above the threshold is missing"
     assert not np.any(sel[s < tau]), "an element below the threshold is selected"
     assert sel[s == tau].sum() == kt - np.count_nonzero(s > tau)
+
+
+# ------------------------------------------------------------------ full-size checks in a process pool
+def oracle_pool(workers=None):
+    """Process pool for oracle work at full size.  Started with spawn, so that
+    it is safe after the parent has used the GPU."""
+    import multiprocessing
+    import os
+    from concurrent.futures import ProcessPoolExecutor
+    n = workers or max(1, min(32, os.cpu_count() or 1))
+    return ProcessPoolExecutor(max_workers=n, mp_context=multiprocessing.get_context("spawn"))
+
+
+def _one_thread():
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except Exception:
+        pass
+
+
+def oracle_seq_cache(task):
+    """Worker: one sequence's oracle cache (prior keys, then this call's keys).
+    task = (k_prior bits [p,128], k_new bits [n,128], T_cap, fmt); returns
+    (codes [p+n,128], scales [p+n])."""
+    _one_thread()
+    k_prior, k_new, T_cap, fmt = task
+    p, n = k_prior.shape[0], k_new.shape[0]
+    kc = np.zeros((1, p + n, 128), np.uint8)
+    ks = np.zeros((1, p + n), np.float32)
+    if p:
+        O.quant_append(k_prior[None], [0], kc, ks, fmt)
+    O.quant_append(k_new[None], [p], kc, ks, fmt)
+    return kc[0], ks[0]
+
+
+def oracle_check_rows(task):
+    """Worker: the oracle's scores of some rows of one sequence, then the
+    top-k set check of the GPU's rows.  task = (q codes [R,64,128], w [R,64],
+    cache codes, scales, visible counts [R], GPU indices [R,k], k, row ids).
+    Returns the number of rows checked."""
+    _one_thread()
+    qc, w, kc, ks, vis, got, k, rows = task
+    S, E = O.index_scores_rows(qc, w, kc, ks, vis)
+    for r in range(len(vis)):
+        try:
+            check_topk_row(got[r], S[r], E[r], int(vis[r]), k)
+        except AssertionError as e:
+            raise AssertionError(f"row {rows[r]}: {e}") from None
+    return len(vis)

@@ -432,6 +432,30 @@ def test_scores_odd_in_weights_and_linear_when_logits_positive():
     assert np.all(np.abs(Sab[m] - (Sa[m] + Sb[m])) <= tol)
 
 
+def test_batched_row_scores_equal_the_per_row_definition():
+    """index_scores_rows (matrix products over all rows and heads) against
+    index_scores (one row at a time): the logits are exact in both, so only
+    the float64 order of the 64-term head sums may differ."""
+    case = synth.make_case("rows", 91, 2, 37, [300, 45], T_cap=512, causal=True, fmt=1)
+    kc, ks = np.zeros((2, 512, 128), np.uint8), np.zeros((2, 512), np.float32)
+    for b in range(2):
+        p = int(case.positions[b])
+        O.quant_append(case.k_prior[b:b + 1, :p], [0], kc[b:b + 1], ks[b:b + 1], 1)
+    O.quant_append(case.k_new, case.positions, kc, ks, 1)
+    qc, _, w = O.quant_queries(case.q, case.w_raw, 1)
+    for causal in (True, False):
+        S, E = O.index_scores(qc, w, kc, ks, case.lengths, causal, ncols=int(case.lengths.max()))
+        for b in range(2):
+            L = int(case.lengths[b])
+            vis = [O.visible_count(L, 37, i, causal) for i in range(37)]
+            S2, E2 = O.index_scores_rows(qc[b], w[b], kc[b], ks[b], vis)
+            V = max(vis)
+            assert np.array_equal(np.isneginf(S2), np.isneginf(S[b, :, :V]))
+            fin = ~np.isneginf(S2)
+            assert np.all(np.abs(S2[fin] - S[b, :, :V][fin]) <= 1e-13 * E[b, :, :V][fin])
+            assert np.allclose(E2, E[b, :, :V], rtol=1e-13, atol=0)
+
+
 def test_causal_visibility_rule():
     qc, w, kc, ks, _, _ = _rand_case(34, B=1, n=4, T=10, lengths=(10,))
     S, _ = O.index_scores(qc, w, kc, ks, np.array([10]), True, ncols=10)

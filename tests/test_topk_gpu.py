@@ -85,8 +85,8 @@ FUSED = [
     ("decode-small-k", 4, 1, [511, 2000, 777, 3333], 4096, False, 0, 17),
     ("prefill", 1, 300, [0], 512, True, 0, 64),
     ("chunked", 2, 130, [900, 2500], 4096, True, 1, 512),
-    # 64 decode rows: with a workspace the scorer splits rows over plain CTAs
-    # and the top-k takes one row per CTA
+    # 64 decode rows, fewer than the SMs: the fused kernel splits each row over
+    # a cluster of 2 CTAs that select through distributed shared memory
     ("decode-many", 64, 1, list(range(1000, 2024, 16)), 2048, False, 1, 256),
 ]
 
@@ -102,9 +102,8 @@ def test_fused_topk_matches_oracle_and_unfused(name, B, n, positions, T_cap, cau
     ws = None
     if use_ws:
         nbytes = X.workspace_size(B, n, max_len, k)
-        if nbytes == 0:
-            pytest.skip("decode-shaped calls use no workspace")
-        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        # a decode-shaped call needs none: one offered anyway must leave the result as it is
+        ws = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device="cuda")
     idx = X.score_topk(qc, w, kc, ks, lengths, causal, k, max_len, ws=ws).cpu().numpy()
     sc = X.score(qc, w, kc, ks, lengths, causal, max_len, ld=max_len).cpu().numpy()
     assert X.status() == (0, 0)

@@ -78,3 +78,31 @@ def test_noalloc_rejects_calls_beyond_its_scratch():
     assert code == -10
     assert b"scratch" in lib.idx_error_string(code)
     assert X.status() == (0, 0)
+
+
+
+def test_noalloc_first_call_decode_shaped_then_prefill_allocates_nothing():
+    """The first call here is decode-shaped: in a fresh process it is the call
+    that looks up the fixed buffer's address, whatever its shape.  A
+    prefill-shaped call after it must still match the workspace path, and a
+    call leaves the device's free memory exactly as it was (no allocation)."""
+    from sparse_attention_token_idx_b200 import binding as X
+    lib = X.load()
+    dec = _prepare("decode", 3, 1, [1000, 77, 3000], 4096, False, 0, 256)
+    got_dec = _noalloc(X, *dec)
+    _same_sets(got_dec, _with_workspace(X, *dec))
+    case, kc, ks, lengths, qc, w = _prepare(*CASES[1])
+    ref = _with_workspace(X, case, kc, ks, lengths, qc, w)
+    max_len = int(case.lengths.max())
+    out = torch.full((case.B, case.n, case.k), -7, dtype=torch.int32, device="cuda")
+    args = (qc.data_ptr(), w.data_ptr(), kc.data_ptr(), ks.data_ptr(), lengths.data_ptr(), case.B, case.n, case.T_cap,
+            max_len, int(case.causal), case.k, out.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    for _ in range(2):
+        out.fill_(-7)
+        torch.cuda.synchronize()
+        free0 = torch.cuda.mem_get_info()[0]
+        assert lib.idx_score_topk_noalloc(*args) == 0
+        torch.cuda.synchronize()
+        assert torch.cuda.mem_get_info()[0] == free0
+        _same_sets(out.cpu().numpy(), ref)
+    assert X.status() == (0, 0)
