@@ -371,22 +371,27 @@ def oracle_step_timer(case, seqs, key_limit=None):
     return run, keys
 
 
-def cpu_baseline(case, target_s=8.0, max_seqs=64):
-    """Time the oracle on a bounded sample of the workload, scaled to keys/s."""
-    seqs = [0]
-    run, keys = oracle_step_timer(case, seqs)
+def cpu_baseline(case, target_s=12.0):
+    """Time the oracle on a bounded sample of the workload, scaled to keys/s:
+    whole oracle steps (append, quantise queries, fp64 scores, full-sort top-k)
+    over as many sequences as fit about target_s of CPU time, repeated until
+    that much time has passed."""
+    run, keys = oracle_step_timer(case, [0])
     t = time.perf_counter()
     run()
-    one = time.perf_counter() - t
-    nseq = int(max(1, min(case.B, max_seqs, target_s / max(one, 1e-3))))
+    one = max(time.perf_counter() - t, 1e-4)
+    nseq = int(max(1, min(case.B, target_s / 2 / one)))
+    seqs = list(range(nseq))
     if nseq > 1:
-        seqs = list(range(nseq))
         run, keys = oracle_step_timer(case, seqs)
+    reps, dt = 0, 0.0
     t = time.perf_counter()
-    run()
-    dt = time.perf_counter() - t
-    return {"value": keys / dt, "unit": "keys/s", "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"{len(seqs)} of {case.B} sequences of '{case.name}', one full oracle step "
+    while reps == 0 or dt < target_s:
+        run()
+        reps += 1
+        dt = time.perf_counter() - t
+    return {"value": keys * reps / dt, "unit": "keys/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{len(seqs)} of {case.B} sequences of '{case.name}', {reps} full oracle steps "
                       f"(append, quantise queries, fp64 scores, full-sort top-{case.k}) in {dt:.1f} s"}
 
 

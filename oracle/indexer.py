@@ -29,6 +29,9 @@ What it computes, step by step, with the passage each step follows:
 * ``topk``             — ``Indexer.forward`` excerpt (top min(index_topk, ·)
   positions per row) and the NKI "DeepSeek-V3.2 Sparse Indexer Kernel API
   Reference" page, Notes and return types (int32, an unordered set).
+* ``project`` — the three projections that open the ``Indexer.forward``
+  excerpt (wq_b of the low-rank query, wk of the hidden state, weights_proj
+  of the hidden state in fp32).
 * ``layer_norm_bf16``, ``rope_bf16``, ``front`` — the steps before the
   rotation in the ``Indexer.forward`` excerpt: the key LayerNorm (k_norm), and
   the rotary embedding, not interleaved, of the queries and keys (gain and
@@ -64,6 +67,10 @@ Readings taken where the pages are silent:
   heads, "Join query parts" page); not interleaved means feature i pairs with
   i + 32.  The angles come in as cos / sin tables (NKI page), so the YaRN
   frequency schedule is outside this step.
+* The projections' weights: wq_b and wk bf16 in the Linear layout [out, in]
+  (the excerpt calls them as Linear layers and gives no dtype; the NKI page's
+  MX-fp8 wq_b is a Trainium packing), weights_proj fp32 (the excerpt casts
+  x to fp32 before it).  Outputs rounded once, to bf16 (q, k) and fp32 (w).
 * LayerNorm: biased variance, eps added under the square root, all in float64
   with sums taken from feature 0 to 127; its output is bf16 (the activations'
   type), and so is the RoPE output.  eps is an argument (fp32).
@@ -286,6 +293,31 @@ def rope_bf16(x_bf16_bits, cos, sin):
     y[..., :half] = a * c - b * s
     y[..., half:ROPE_DIM] = b * c + a * s
     return f64_to_bf16_bits(bf16_round(y))
+
+
+def project(x_bits, qr_bits, wq_b_bits, wk_bits, w_proj):
+    """The indexer's three projections, the first steps of the Indexer.forward
+    excerpt ("Index scores" page): q = wq_b(qr) viewed as [tokens, 64, 128]
+    (head-major), k = wk(x), and the head weights weights_proj(x.float()).
+
+    x [T, hidden] and qr [T, q_lora] bf16 bits; wq_b [64·128, q_lora] and
+    wk [128, hidden] bf16 bits (Linear layout: [out, in]); w_proj [64, hidden]
+    float32.  Each product is a float64 matrix product of the exact inputs
+    (every bf16 × bf16 or bf16 × fp32 product is exact in float64, and the
+    sums stay within one float64 rounding per term), then ONE rounding: to
+    bf16 for q and k (the activations' type), to fp32 for the weights (the
+    excerpt's x.float()).  Returns (q [T, 64, 128] bf16 bits, k [T, 128] bf16
+    bits, w_raw [T, 64] float32)."""
+    x = bf16_bits_to_f64(x_bits)
+    qr = bf16_bits_to_f64(qr_bits)
+    wq = bf16_bits_to_f64(wq_b_bits)
+    wk = bf16_bits_to_f64(wk_bits)
+    wp = np.asarray(w_proj, np.float32).astype(np.float64)
+    T = x.shape[0]
+    q = f64_to_bf16_bits(bf16_round(qr @ wq.T)).reshape(T, H, D)
+    k = f64_to_bf16_bits(bf16_round(x @ wk.T))
+    w = (x @ wp.T).astype(np.float32)
+    return q, k, w
 
 
 def front(q_proj_bits, k_proj_bits, cos, sin, gain, bias, eps):

@@ -28,6 +28,7 @@
 #include <cstdint>
 
 #include "api_internal.h"
+#include "epilogue.cuh"
 #include "ptx.cuh"
 
 namespace idx {
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(FCfg<NT, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W
     // W_REGS: this warp's 64 head weights (one row) in registers, packed in
     // pairs for the f32x2 FMA, reloaded per row block; otherwise they are read
     // from shared memory (broadcast 16-byte loads) to stay within the registers
-    static_assert(!W_REGS || C::kTokPerWarp == 1, "register weights hold one row");
+    static_assert(C::kTokPerWarp == 1, "one query row per epilogue warp");
     unsigned long long wp[W_REGS ? 32 : 1];
     if (nunits > 0) {
       Walker wk;
@@ -341,59 +342,16 @@ __global__ void __launch_bounds__(FCfg<NT, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W
                                       : scale_s[c * kFKeys + kl];
           const int key = wk.tile * kFKeys + kl;
           const float* wrow = w_s + (qseq & 1) * N;
-#pragma unroll
-          for (int jj = 0; jj < C::kTokPerWarp; ++jj) {
-            const int j = tok_lo + jj;
-            unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
-            if constexpr (W_REGS) {
-              // both halves of the row's 64 logits in flight before one wait
-              uint32_t r0[32], r1[32];
-              tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64), r0);
-              tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64 + 32), r1);
-              tmem_wait();
-              tmem_regs_ready(r0);
-              tmem_regs_ready(r1);
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                fma2(acc[i & 3],
-                     pack2(fmaxf(__uint_as_float(r0[2 * i]), 0.f), fmaxf(__uint_as_float(r0[2 * i + 1]), 0.f)),
-                     wp[i]);
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                fma2(acc[i & 3],
-                     pack2(fmaxf(__uint_as_float(r1[2 * i]), 0.f), fmaxf(__uint_as_float(r1[2 * i + 1]), 0.f)),
-                     wp[16 + i]);
-            } else {
-              // both halves in flight before one wait; weights from shared memory
-              uint32_t r[2][32];
-              tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64), r[0]);
-              tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64 + 32), r[1]);
-              tmem_wait();
-              tmem_regs_ready(r[0]);
-              tmem_regs_ready(r[1]);
-#pragma unroll
-              for (int c = 0; c < 2; ++c) {
-                const float4* wv = reinterpret_cast<const float4*>(wrow + j * 64 + c * 32);
-#pragma unroll
-                for (int i4 = 0; i4 < 8; ++i4) {
-                  const float4 w4 = wv[i4];
-                  fma2(acc[(2 * i4) & 3],
-                       pack2(fmaxf(__uint_as_float(r[c][4 * i4]), 0.f), fmaxf(__uint_as_float(r[c][4 * i4 + 1]), 0.f)),
-                       pack2(w4.x, w4.y));
-                  fma2(acc[(2 * i4 + 1) & 3],
-                       pack2(fmaxf(__uint_as_float(r[c][4 * i4 + 2]), 0.f),
-                             fmaxf(__uint_as_float(r[c][4 * i4 + 3]), 0.f)),
-                       pack2(w4.z, w4.w));
-                }
-              }
-            }
-            const float2 p0 = unpack2(acc[0]), p1 = unpack2(acc[1]), p2 = unpack2(acc[2]), p3 = unpack2(acc[3]);
-            const float sc = (((p0.x + p0.y) + (p1.x + p1.y)) + ((p2.x + p2.y) + (p3.x + p3.y))) * ks;
-            const int row = blk.row0 + j;
-            if (row < p.n && key < p.ld)
-              p.scores[(static_cast<int64_t>(blk.b) * p.n + row) * p.ld + key] = key < blk.vis(p, row) ? sc
-                                                                                                     : -INFINITY;
-          }
+          uint32_t r[64];
+          load_logits(lane_base + static_cast<uint32_t>(a * N + tok_lo * 64), r);
+          float sc;
+          if constexpr (W_REGS) sc = relu_head_sum(r, wp, ks);
+          else sc = relu_head_sum(r, wrow + tok_lo * 64, ks);
+          const int row = blk.row0 + tok_lo;
+          if (row < p.n && key < p.ld)
+            p.scores[(static_cast<int64_t>(blk.b) * p.n + row) * p.ld + key] = key < blk.vis(p, row) ? sc : -INFINITY;
+          // the accumulator and the scale slot go back after the arithmetic
+          // (handing them back right after the TMEM load measured slower)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) {

@@ -27,6 +27,7 @@
 #include <mutex>
 
 #include "api_internal.h"
+#include "epilogue.cuh"
 #include "ptx.cuh"
 #include "select.cuh"
 
@@ -155,6 +156,47 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
   const int b = item % p.B;
   const int tb = p.ntb - 1 - item / p.B;   // longest (latest) row blocks first
   const int row0 = tb * NT;
+  int tma_issued = 0;     // producer lane (thread 0): K tiles whose loads were issued
+  bool q_issued = false;  // producer lane: the query load was issued
+  // Thread 0 is also the TMA producer: it starts the query and the first
+  // STAGES key tiles during the set-up, so that their DRAM latency overlaps it
+  // (the ring is empty, no slot needs to be waited for).
+  auto issue_first = [&](int tiles, int start0) {
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_s);
+    mbar_arrive_expect_tx(q_full, C::kQBytes);
+    tma_load_3d(q_s, &tmap_q, q_full, 0, row0 * IDX_HEADS, b);
+    q_issued = true;
+    const int pre = tiles < STAGES ? tiles : STAGES;
+    for (int t = 0; t < pre; ++t) {
+      mbar_arrive_expect_tx(&full[t], kTileBytes + kTileKeys * (p.scale_u8 ? 1 : 4));
+      tma_load_3d(k_s + t * kTileBytes, &tmap_k, &full[t], 0, start0 + t * kTileKeys, b);
+      tma_load_2d(scale_s + t * kTileKeys, &tmap_s, &full[t], start0 + t * kTileKeys, b);
+    }
+    tma_issued = pre;
+  };
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);   // the MMA is done with the keys
+    }
+    for (int c = 0; c < C::kScaleSlots; ++c) mbar_init(&sc_empty[c], C::kWarpsPerTile);   // epilogue done with the scales
+    for (int a = 0; a < NUM_ACC; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], C::kWarpsPerTile);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(drain_bar, 1);
+    mbar_init(never_bar, 1);
+    *abort_flag = 0;
+    if constexpr (FUSED) row_filter_reset(sel.cta);
+    fence_barrier_init();
+    // one CTA per row block: the slice starts at key 0 and the host bound
+    // max_len sizes the first requests, so they leave before lengths[b] has
+    // arrived; tiles past the row's keys are drained at the end like any other
+    if (G == 1) issue_first(ceil_div(p.max_len, kTileKeys), 0);
+  }
   const int len = p.lengths[b];
   const bool bad = len < p.n || len > p.max_len;
   if (bad && rank == 0 && threadIdx.x == 0) raise_error(p.err, IDX_DEV_ERR_LENGTH);
@@ -173,50 +215,15 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
   const int end = min(start + chunk, vis_max);
   const int ntiles = end > start ? ceil_div(end - start, kTileKeys) : 0;
   auto tile_of = [](int t) { return t; };   // tiles are visited in order
-
-  int tma_issued = 0;     // producer lane (thread 0): K tiles whose loads were issued
-  bool q_issued = false;  // producer lane: the query load was issued
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);   // the MMA is done with the keys
-    }
-    for (int c = 0; c < C::kScaleSlots; ++c) mbar_init(&sc_empty[c], C::kWarpsPerTile);   // epilogue done with the scales
-    for (int a = 0; a < NUM_ACC; ++a) {
-      mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], C::kWarpsPerTile);
-    }
-    mbar_init(q_full, 1);
-    mbar_init(drain_bar, 1);
-    mbar_init(never_bar, 1);
-    *abort_flag = 0;
-    if constexpr (FUSED) row_filter_reset(sel.cta);
-    fence_barrier_init();
-    // Thread 0 is also the TMA producer: start the query and the first STAGES
-    // key tiles now, so that their DRAM latency overlaps the rest of the set-up
-    // (the ring is empty, no slot needs to be waited for).
-    if (ntiles > 0) {
-      tma_prefetch_desc(&tmap_k);
-      tma_prefetch_desc(&tmap_q);
-      tma_prefetch_desc(&tmap_s);
-      mbar_arrive_expect_tx(q_full, C::kQBytes);
-      tma_load_3d(q_s, &tmap_q, q_full, 0, row0 * IDX_HEADS, b);
-      q_issued = true;
-      const int pre = ntiles < STAGES ? ntiles : STAGES;
-      for (int t = 0; t < pre; ++t) {
-        mbar_arrive_expect_tx(&full[t], kTileBytes + kTileKeys * (p.scale_u8 ? 1 : 4));
-        const int tt = tile_of(t);
-        tma_load_3d(k_s + t * kTileBytes, &tmap_k, &full[t], 0, start + tt * kTileKeys, b);
-        tma_load_2d(scale_s + t * kTileKeys, &tmap_s, &full[t], start + tt * kTileKeys, b);
-      }
-      tma_issued = pre;
-    }
-  }
+  // a slice of a split row starts where this CTA's share does
+  if (G > 1 && threadIdx.x == 0 && ntiles > 0) issue_first(ntiles, start);
   if (warp == 1) tmem_alloc(tmem_slot, C::kTmemCols);
   for (int i = threadIdx.x; i < N; i += blockDim.x) {
     const int j = i / IDX_HEADS;
     const int tok = row0 + j;
-    w_s[i] = (tok < p.n && !bad) ? p.w[(static_cast<int64_t>(b) * p.n + tok) * IDX_HEADS + (i % IDX_HEADS)] : 0.f;
+    // not gated on the length check (a bad length masks every key anyway), so
+    // that this load overlaps the one of lengths[b]
+    w_s[i] = tok < p.n ? p.w[(static_cast<int64_t>(b) * p.n + tok) * IDX_HEADS + (i % IDX_HEADS)] : 0.f;
   }
   if constexpr (FUSED) {
     for (int i = threadIdx.x; i < NT * kHistBins; i += blockDim.x) hist1[i] = 0;
@@ -286,7 +293,7 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
     // W_REGS: this warp's 64 head weights (one row) in registers, packed in
     // pairs for the f32x2 FMA; otherwise they are read from shared memory
     // (broadcast 16-byte loads) to stay within the register budget.
-    static_assert(!W_REGS || C::kTokPerWarp == 1, "register weights hold one row");
+    static_assert(C::kTokPerWarp == 1, "one query row per epilogue warp");
     unsigned long long wp[W_REGS ? 32 : 1];
     if constexpr (W_REGS) {
 #pragma unroll
@@ -308,66 +315,29 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
       const float ks = p.scale_u8 ? __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint8_t*>(
                                         scale_s + sc_slot * kTileKeys)[kl]) << 23)
                                   : scale_s[sc_slot * kTileKeys + kl];
-#pragma unroll
-      for (int jj = 0; jj < C::kTokPerWarp; ++jj) {
-        const int j = tok_lo + jj;
-        unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
-        if constexpr (W_REGS) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64), r0);
-          tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64 + 32), r1);
-          tmem_wait();
-          tmem_regs_ready(r0);
-          tmem_regs_ready(r1);
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            fma2(acc[i & 3], pack2(fmaxf(__uint_as_float(r0[2 * i]), 0.f), fmaxf(__uint_as_float(r0[2 * i + 1]), 0.f)),
-                 wp[i]);
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            fma2(acc[i & 3], pack2(fmaxf(__uint_as_float(r1[2 * i]), 0.f), fmaxf(__uint_as_float(r1[2 * i + 1]), 0.f)),
-                 wp[16 + i]);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t r0[32];
-            tmem_ld32_nowait(lane_base + static_cast<uint32_t>(a * N + j * 64 + c * 32), r0);
-            tmem_wait();
-            tmem_regs_ready(r0);
-            const float4* wv = reinterpret_cast<const float4*>(w_s + j * 64 + c * 32);
-#pragma unroll
-            for (int i4 = 0; i4 < 8; ++i4) {
-              const float4 w4 = wv[i4];
-              fma2(acc[(2 * i4) & 3],
-                   pack2(fmaxf(__uint_as_float(r0[4 * i4]), 0.f), fmaxf(__uint_as_float(r0[4 * i4 + 1]), 0.f)),
-                   pack2(w4.x, w4.y));
-              fma2(acc[(2 * i4 + 1) & 3],
-                   pack2(fmaxf(__uint_as_float(r0[4 * i4 + 2]), 0.f), fmaxf(__uint_as_float(r0[4 * i4 + 3]), 0.f)),
-                   pack2(w4.z, w4.w));
-            }
-          }
+      const int j = tok_lo;
+      uint32_t r[64];
+      load_logits(lane_base + static_cast<uint32_t>(a * N + j * 64), r);
+      float sc;
+      if constexpr (W_REGS) sc = relu_head_sum(r, wp, ks);
+      else sc = relu_head_sum(r, w_s + j * 64, ks);
+      const bool visible = key < row_vis(j);
+      if constexpr (FUSED) {
+        const uint32_t u = order_key(sc);
+        sc_s[j * p.chunk_cap + tt * kTileKeys + kl] = visible ? u : 0u;
+        if (visible) {
+          if constexpr (NT == 1) select_count_key(sel.cta, hist1, u);   // with the coarse sums
+          else atomicAdd(&hist1[j * kHistBins + (u >> 21)], 1u);
         }
-        const float2 p0 = unpack2(acc[0]), p1 = unpack2(acc[1]), p2 = unpack2(acc[2]), p3 = unpack2(acc[3]);
-        const float part[4] = {p0.x + p0.y, p1.x + p1.y, p2.x + p2.y, p3.x + p3.y};
-        const float sc = ((part[0] + part[1]) + (part[2] + part[3])) * ks;
-        const bool visible = key < row_vis(j);
-        if constexpr (FUSED) {
-          const uint32_t u = order_key(sc);
-          sc_s[j * p.chunk_cap + tt * kTileKeys + kl] = visible ? u : 0u;
-          if (visible) {
-            if constexpr (NT == 1) select_count_key(sel.cta, hist1, u);   // with the coarse sums
-            else atomicAdd(&hist1[j * kHistBins + (u >> 21)], 1u);
-          }
-          // one row per CTA: keys that may reach the top k go to the short list
-          if constexpr (C::kList > 0)
-            if (G == 1) row_filter_append(sel.cta, list16, C::kList, u, visible, tt * kTileKeys + kl);
-        } else {
-          if (row_exists(j) && key < p.ld) {
-            const int64_t at = (static_cast<int64_t>(b) * p.n + row0 + j) * p.ld + key;
-            const float v = visible ? sc : p.mask_value;
-            if (p.out_bf16) static_cast<__nv_bfloat16*>(p.scores)[at] = __float2bfloat16_rn(v);
-            else static_cast<float*>(p.scores)[at] = v;
-          }
+        // one row per CTA: keys that may reach the top k go to the short list
+        if constexpr (C::kList > 0)
+          if (G == 1) row_filter_append(sel.cta, list16, C::kList, u, visible, tt * kTileKeys + kl);
+      } else {
+        if (row_exists(j) && key < p.ld) {
+          const int64_t at = (static_cast<int64_t>(b) * p.n + row0 + j) * p.ld + key;
+          const float v = visible ? sc : p.mask_value;
+          if (p.out_bf16) static_cast<__nv_bfloat16*>(p.scores)[at] = __float2bfloat16_rn(v);
+          else static_cast<float*>(p.scores)[at] = v;
         }
       }
       tc_fence_before();

@@ -106,3 +106,30 @@ def workload(idx: int) -> Case:
     if idx == 4:
         return make_case(name, seed, 2, 2048, [14336, 14336], causal=True, fmt=1)
     raise KeyError(idx)
+
+
+# --------------------------------------------------------------------------- projections
+HIDDEN = 7168          # hidden width of the synthetic projections (a multiple of 128)
+Q_LORA = 1536          # low-rank query width (a multiple of 512, the NKI page's MX K-tile)
+
+
+@dataclass
+class ProjCase:
+    x: np.ndarray          # uint16 bf16 bits [T, hidden]
+    qr: np.ndarray         # uint16 bf16 bits [T, q_lora]
+    wq_b: np.ndarray       # uint16 bf16 bits [64·128, q_lora]  (Linear layout [out, in])
+    wk: np.ndarray         # uint16 bf16 bits [128, hidden]
+    w_proj: np.ndarray     # float32 [64, hidden]
+
+
+def make_proj_case(seed, tokens, hidden=HIDDEN, q_lora=Q_LORA) -> ProjCase:
+    """Random projection inputs and weights: x, qr ~ N(0, 1); each weight
+    matrix ~ N(0, 1 / fan_in) so that the outputs are O(1).  Drawn in this
+    order with NumPy PCG64(seed): x, qr, wq_b, wk, w_proj."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    x = rng.standard_normal((tokens, hidden), dtype=np.float32)
+    qr = rng.standard_normal((tokens, q_lora), dtype=np.float32)
+    wq = rng.standard_normal((H * D, q_lora), dtype=np.float32) / np.float32(np.sqrt(q_lora))
+    wk = rng.standard_normal((D, hidden), dtype=np.float32) / np.float32(np.sqrt(hidden))
+    wp = rng.standard_normal((H, hidden), dtype=np.float32) / np.float32(np.sqrt(hidden))
+    return ProjCase(_to_bf16_bits(x), _to_bf16_bits(qr), _to_bf16_bits(wq), _to_bf16_bits(wk), wp.astype(np.float32))

@@ -700,3 +700,33 @@ def test_front_orders_layer_norm_before_rope_and_leaves_weights_alone():
         assert np.array_equal(fq[t], O.rope_bf16(q[t], c[t], s[t]))
     assert np.array_equal(fk, O.rope_bf16(O.layer_norm_bf16(k, g, b, 1e-6), c, s))
     assert not np.array_equal(fk, O.layer_norm_bf16(O.rope_bf16(k, c, s), g, b, 1e-6))
+
+
+# --------------------------------------------------------------------------- projections
+def test_projections_match_torch_and_exact_rounding():
+    """project() against torch's float64 matmul on the same exact inputs (the
+    bf16 outputs must agree), the head-major view of q pinned by one-hot
+    weights (output h·128 + d lands in head h, feature d), and a few outputs
+    recomputed in exact rationals then rounded once."""
+    pc = synth.make_proj_case(5, 9, hidden=256, q_lora=512)
+    q, k, w = O.project(pc.x, pc.qr, pc.wq_b, pc.wk, pc.w_proj)
+    assert q.shape == (9, 64, 128) and k.shape == (9, 128) and w.shape == (9, 64) and w.dtype == np.float32
+    tx = torch.from_numpy(O.bf16_bits_to_f64(pc.x))
+    tq = torch.from_numpy(O.bf16_bits_to_f64(pc.qr))
+    tq_ref = tq @ torch.from_numpy(O.bf16_bits_to_f64(pc.wq_b)).T
+    tk_ref = tx @ torch.from_numpy(O.bf16_bits_to_f64(pc.wk)).T
+    np.testing.assert_array_equal(q.reshape(9, -1), O.f64_to_bf16_bits(O.bf16_round(tq_ref.numpy())))
+    np.testing.assert_array_equal(k, O.f64_to_bf16_bits(O.bf16_round(tk_ref.numpy())))
+    tw = (tx @ torch.from_numpy(pc.w_proj.astype(np.float64)).T).numpy().astype(np.float32)
+    np.testing.assert_array_equal(w.view(np.uint32), tw.view(np.uint32))
+    # exact rationals for a handful of outputs
+    xs = O.bf16_bits_to_f64(pc.qr)
+    ws = O.bf16_bits_to_f64(pc.wq_b)
+    for t, o in ((0, 0), (3, 4097), (8, 8191)):
+        exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(xs[t], ws[o]))
+        assert Fraction(float(O.bf16_bits_to_f64(q.reshape(9, -1)[t, o]))) == bf16_exact(exact)
+    # head-major layout: a weight row that copies qr feature 0 into output h·128 + d
+    wq1 = np.zeros((64 * 128, 512), np.uint16)
+    wq1[5 * 128 + 17, 0] = 0x3F80                    # 1.0 in bf16
+    q1, _, _ = O.project(pc.x, pc.qr, wq1, pc.wk, pc.w_proj)
+    assert np.array_equal(q1[:, 5, 17], pc.qr[:, 0]) and np.count_nonzero(q1) == np.count_nonzero(pc.qr[:, 0])
