@@ -7,8 +7,9 @@
  *   scores:  S[t,s] = k_scale[s] · Σ_{h<64} w[t,h] · ReLU(q_fp8[t,h] · k_fp8[s]);
  *   select:  the min(k, visible) highest-scoring cached positions per query row.
  *
- * Around that path: the front end before it (query RoPE, key LayerNorm + RoPE,
- * fused with the quantiser: idx_front_quant_append), the attention after it
+ * Around that path: the front end before it (the three projections on the
+ * tensor cores: idx_project; query RoPE, key LayerNorm + RoPE, fused with the
+ * quantiser: idx_front_quant_append), the attention after it
  * (sparse latent attention over the selected positions: idx_sparse_mla_decode),
  * and split-T selection of one sequence over several GPUs (idx_gather_scores,
  * idx_merge_topk).
@@ -186,6 +187,30 @@ IDX_API int idx_front_quant_append(const uint16_t* q_proj, const float* w_raw, c
                                    const float* ln_bias, float ln_eps, const int32_t* positions, int B, int n,
                                    uint8_t* q_fp8, float* w, uint8_t* k_cache, float* k_scale_cache, int T_cap,
                                    int fmt, idx_stream_t stream);
+
+/*
+ * idx_project — the three projections that open the Indexer.forward excerpt
+ * ("Index scores" page): q = wq_b(qr) viewed as 64 heads of 128 features,
+ * k = wk(x), and the head weights weights_proj(x.float()).
+ *   x      [tokens, hidden] bf16 (hidden a multiple of 128), the hidden state.
+ *   qr     [tokens, q_lora] bf16 (q_lora a multiple of 64), the low-rank query.
+ *   wq_b   [64·128, q_lora] bf16, wk [128, hidden] bf16: Linear weights [out, in].
+ *   w_proj [64, hidden] fp32.
+ *   q_proj [tokens, 64, 128] bf16 out, k_proj [tokens, 128] bf16 out: the fp32
+ *          products (tensor cores, fp32 accumulation) rounded to nearest-even bf16;
+ *          ready for idx_front_quant_append.
+ *   w_raw  [tokens, 64] fp32 out: Σ_k x·w_proj in fp32, k ascending (CUDA cores).
+ *   ws / ws_bytes: scratch of idx_project_workspace_size(tokens, hidden, q_lora)
+ *          bytes (16-byte aligned) for the fp32 partial sums of a product split
+ *          over K when few tokens cannot fill the GPU; a smaller workspace (or
+ *          none) means fewer splits, never an error.
+ * All bf16 pointers and ws must be 16-byte aligned.  Errors: IDX_ERR_SHAPE,
+ * IDX_ERR_NULL, IDX_ERR_ALIGN.
+ */
+IDX_API size_t idx_project_workspace_size(int64_t tokens, int hidden, int q_lora);
+IDX_API int idx_project(const uint16_t* x, const uint16_t* qr, int64_t tokens, int hidden, int q_lora,
+                        const uint16_t* wq_b, const uint16_t* wk, const float* w_proj, uint16_t* q_proj,
+                        uint16_t* k_proj, float* w_raw, void* ws, size_t ws_bytes, idx_stream_t stream);
 
 /*
  * idx_score — "Index scores" page: score equation and fp8_index docstring

@@ -54,6 +54,8 @@ SIGNATURES = {
     "idx_score_topk_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P]),
     "idx_score_topk_ex": (_I, [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "idx_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "idx_project": (_I, [_P, _P, _I64, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "idx_project_workspace_size": (_SZ, [_I64, _I, _I]),
     "idx_status": (_I, [_P]),
     "idx_device_error_bits": (ctypes.c_uint, []),
     "idx_error_string": (ctypes.c_char_p, [_I]),
@@ -177,6 +179,37 @@ def front_quant_append(q_proj, w_raw, k_proj, rope_cos, rope_sin, ln_gain, ln_bi
         _ptr(k_scale_cache, torch.float32, "k_scale_cache"), k_cache.shape[1], fmt, _stream(stream)),
         "idx_front_quant_append")
     return q_out, w_out
+
+
+def project_workspace_size(tokens: int, hidden: int, q_lora: int) -> int:
+    return int(load().idx_project_workspace_size(tokens, hidden, q_lora))
+
+
+def project(x, qr, wq_b, wk, w_proj, q_out=None, k_out=None, w_out=None, ws=None, stream=None):
+    """The three projections: x [T, hidden] bf16, qr [T, q_lora] bf16, wq_b
+    [64·128, q_lora] bf16, wk [128, hidden] bf16, w_proj [64, hidden] fp32 →
+    (q_proj [T, 64, 128] bf16, k_proj [T, 128] bf16, w_raw [T, 64] fp32).
+    ws: uint8 workspace of project_workspace_size bytes (allocated when None)."""
+    T, hidden = x.shape
+    q_lora = qr.shape[1]
+    if tuple(qr.shape) != (T, q_lora) or tuple(wq_b.shape) != (HEADS * DIM, q_lora) or \
+            tuple(wk.shape) != (DIM, hidden) or tuple(w_proj.shape) != (HEADS, hidden):
+        raise ValueError("project: x [T, hidden], qr [T, q_lora], wq_b [8192, q_lora], wk [128, hidden], "
+                         "w_proj [64, hidden]")
+    dev = x.device
+    q_out = q_out if q_out is not None else torch.empty((T, HEADS, DIM), dtype=torch.bfloat16, device=dev)
+    k_out = k_out if k_out is not None else torch.empty((T, DIM), dtype=torch.bfloat16, device=dev)
+    w_out = w_out if w_out is not None else torch.empty((T, HEADS), dtype=torch.float32, device=dev)
+    need = project_workspace_size(T, hidden, q_lora)
+    if ws is None and need:
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    _check(load().idx_project(
+        _ptr(x, _BF16, "x"), _ptr(qr, _BF16, "qr"), T, hidden, q_lora, _ptr(wq_b, _BF16, "wq_b"),
+        _ptr(wk, _BF16, "wk"), _ptr(w_proj, torch.float32, "w_proj"), _ptr(q_out, _BF16, "q_out"),
+        _ptr(k_out, _BF16, "k_out"), _ptr(w_out, torch.float32, "w_out"),
+        _ptr(ws, torch.uint8, "ws") if ws is not None else None, ws.numel() if ws is not None else 0,
+        _stream(stream)), "idx_project")
+    return q_out, k_out, w_out
 
 
 def score(q_fp8, w, k_cache, k_scale_cache, lengths, causal: bool, max_len: int, ld: int | None = None,

@@ -167,6 +167,20 @@ bool make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_2d_bf16_sw128(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  resolve_encode();
+  if (!g_encode) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((cols * 2) & 15)) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};   // 64 bf16 = one 128-byte swizzle row
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_scales(CUtensorMap* map, const void* base, int scale_fmt, uint64_t T_cap, uint64_t B,
                       uint32_t box_inner) {
   return scale_fmt == kScaleE8M0 ? make_tmap_u8_2d(map, base, T_cap, B, box_inner)

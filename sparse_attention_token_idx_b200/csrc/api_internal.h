@@ -32,6 +32,10 @@ bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64
 // multiple of 16), box {box_inner, 1}, no swizzle.
 bool make_tmap_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner);
 
+// Tensor map for a [rows, cols] bf16 array (row pitch cols·2 bytes, a multiple
+// of 16), box {64 elements, box_rows}, 128-byte swizzle (K-major MMA operands).
+bool make_tmap_2d_bf16_sw128(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows);
+
 // Key-scale storage of a score call: fp32 values, or e8m0 bytes (2^(byte − 127)).
 enum { kScaleF32 = 0, kScaleE8M0 = 1 };
 

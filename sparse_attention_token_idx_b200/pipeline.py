@@ -85,6 +85,29 @@ class Indexer:
         return X.score_topk_ex(q_fp8, w, self.k_cache, self.k_scale_cache, lengths, causal, self.k, max_len,
                                out=out, ws=ws, stream=stream)
 
+    def step_hidden(self, x, qr, wq_b, wk, w_proj, rope_cos, rope_sin, ln_gain, ln_bias, positions, lengths, *,
+                    causal: bool, max_len: int, ln_eps: float = 1e-6, out=None, stream=None):
+        """One indexer call from the hidden state: x [B, n, hidden] bf16 and qr
+        [B, n, q_lora] bf16 through the projections (wq_b [8192, q_lora], wk
+        [128, hidden] bf16, w_proj [64, hidden] fp32), then as step_front.  The
+        projection outputs stay in this object's buffers (projections())."""
+        B, n = x.shape[0], x.shape[1]
+        T = B * n
+        hidden, q_lora = x.shape[2], qr.shape[2]
+        q_proj = self._buf("q_proj", (B, n, X.HEADS, X.DIM), torch.bfloat16)
+        k_proj = self._buf("k_proj", (B, n, X.DIM), torch.bfloat16)
+        w_raw = self._buf("w_raw", (B, n, X.HEADS), torch.float32)
+        need = X.project_workspace_size(T, hidden, q_lora)
+        ws = self._buf("proj_ws", (need,), torch.uint8)
+        X.project(x.reshape(T, hidden), qr.reshape(T, q_lora), wq_b, wk, w_proj, q_out=q_proj.view(T, X.HEADS, X.DIM),
+                  k_out=k_proj.view(T, X.DIM), w_out=w_raw.view(T, X.HEADS), ws=ws, stream=stream)
+        return self.step_front(q_proj, w_raw, k_proj, rope_cos, rope_sin, ln_gain, ln_bias, positions, lengths,
+                               causal=causal, max_len=max_len, ln_eps=ln_eps, out=out, stream=stream)
+
+    def projections(self):
+        """(q_proj, k_proj, w_raw) of the last step_hidden."""
+        return self._bufs["q_proj"], self._bufs["k_proj"], self._bufs["w_raw"]
+
     def capture(self, k_new, q, w_raw, positions, lengths, *, causal: bool, max_len: int, out=None):
         """Record one step on static input tensors into a CUDA graph; returns
         (graph, out) — replay the graph after refilling the inputs in place.
