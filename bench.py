@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl ours|reference]
                     [--no-prefill] [--no-cpu-baseline]
+    python bench.py --row merge|front|project128|project4096|mla [--steps K] [--warmup W]
 
 A step is one whole indexer call on one batch: append the new keys to the FP8
 cache (rotate + quantise + store), quantise the queries and fold the head
@@ -269,10 +270,28 @@ def measure(args, widx, dev, world, headline):
             ms = sum(a.elapsed_time(b) for a, b in evs)
     if world > 1:
         dist.barrier()
-    # the dominant kernel alone: back-to-back launches between two events
+    # the dominant kernel alone: n_k launches recorded in a CUDA graph (no host
+    # gaps between them) and replayed between two events
     n_k = max(3, min(args.steps, 200))
-    score_ms = back_to_back(score_only, n_k) / n_k
-    topk_ms = back_to_back(topk_only, n_k) / n_k if ws_bytes else None
+
+    def graph_of(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(n_k):
+                fn()
+        return g
+
+    g_score = graph_of(score_only)
+    g_topk = graph_of(topk_only) if ws_bytes else None
+    g_score.replay()
+    torch.cuda.synchronize()
+    score_ms = back_to_back(g_score.replay, 1) / n_k
+    topk_ms = None
+    if g_topk is not None:
+        g_topk.replay()
+        torch.cuda.synchronize()
+        topk_ms = back_to_back(g_topk.replay, 1) / n_k
+    del g_score, g_topk
     code, bits = X.status()
     if code != 0:
         raise RuntimeError(f"device error in the timed region: status {code}, bits {bits}")
@@ -421,6 +440,103 @@ def run_reference(args, rank, world):
     return case, value, dt, sample
 
 
+# ---------------------------------------------------------------------------- widened rows
+ROWS = ("merge", "front", "project128", "project4096", "mla")
+
+
+def row_bench(args, dev, hbm, bf16):
+    """One widened row's launch alone, timed with CUDA events after warm-up, with
+    its algorithmic bytes or FLOPs: the split-T merge (128 rows, 8 × 2048
+    candidates), the fused front end (decode B = 128), the projections (128 and
+    4096 tokens, hidden 7168, q_lora 1536) and the sparse latent attention
+    (B = 128, 128 heads, k = 2048, 16 384 cached positions).  Inputs are random
+    and resident on the device; one L2 flush before the timed launches."""
+    import torch
+    from sparse_attention_token_idx_b200 import binding as X
+    from sparse_attention_token_idx_b200 import synth
+    g = torch.Generator(device=dev).manual_seed(3)
+    row = args.row
+    info = {}
+    if row == "merge":
+        G, rows, kin, k = 8, 128, 2048, 2048
+        sc = torch.randn((G, rows, kin), device=dev, generator=g)
+        pos = torch.stack([torch.randperm(G * kin, device=dev, generator=g).view(G, kin) for _ in range(rows)], 1)
+        cand = torch.stack([sc.view(torch.int32), pos.to(torch.int32)], -1).contiguous()
+        out = torch.empty((rows, k), dtype=torch.int32, device=dev)
+        fn = lambda: X.merge_topk(cand, k, out=out)
+        info = {"bound": "hbm", "algorithmic_bytes": G * rows * kin * 8 + rows * k * 4, "kernel": "merge_topk_kernel",
+                "config": {"rows": rows, "G": G, "kin": kin, "k": k}}
+    elif row == "front":
+        B, T_cap = 128, 16384
+        qp = torch.randn((B, 1, 64, 128), device=dev, generator=g).to(torch.bfloat16)
+        kp = torch.randn((B, 1, 128), device=dev, generator=g).to(torch.bfloat16)
+        wr = torch.randn((B, 1, 64), device=dev, generator=g)
+        ang = torch.rand((B, 1, 32), device=dev, generator=g) * 6.28
+        cos, sin = torch.cos(ang), torch.sin(ang)
+        gain, bias = torch.ones(128, device=dev), torch.zeros(128, device=dev)
+        pos = torch.full((B,), 100, dtype=torch.int32, device=dev)
+        kc = torch.zeros((B, T_cap, 128), dtype=torch.uint8, device=dev)
+        ks = torch.zeros((B, T_cap), dtype=torch.float32, device=dev)
+        q8 = torch.empty((B, 1, 64, 128), dtype=torch.uint8, device=dev)
+        w8 = torch.empty((B, 1, 64), dtype=torch.float32, device=dev)
+        fn = lambda: X.front_quant_append(qp, wr, kp, cos, sin, gain, bias, 1e-6, pos, kc, ks, 0, q_out=q8, w_out=w8)
+        moved = B * (64 * 128 * 2 + 128 * 2 + 64 * 4 + 2 * 32 * 4) + B * (64 * 128 + 64 * 4 + 128 + 4)
+        info = {"bound": "hbm", "algorithmic_bytes": moved, "kernel": "quant_kernel<1> (front end fused)",
+                "config": {"B": B, "n": 1}}
+    elif row in ("project128", "project4096"):
+        T = 128 if row == "project128" else 4096
+        pc = synth.make_proj_case(9, T)
+        bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        x, qr, wq, wk = bf(pc.x), bf(pc.qr), bf(pc.wq_b), bf(pc.wk)
+        wp = torch.from_numpy(pc.w_proj).to(dev)
+        ws = torch.empty(X.project_workspace_size(T, synth.HIDDEN, synth.Q_LORA), dtype=torch.uint8, device=dev)
+        qo = torch.empty((T, 64, 128), dtype=torch.bfloat16, device=dev)
+        ko = torch.empty((T, 128), dtype=torch.bfloat16, device=dev)
+        wo = torch.empty((T, 64), dtype=torch.float32, device=dev)
+        fn = lambda: X.project(x, qr, wq, wk, wp, q_out=qo, k_out=ko, w_out=wo, ws=ws)
+        flops = 2.0 * T * (8192 * synth.Q_LORA + 128 * synth.HIDDEN + 64 * synth.HIDDEN)
+        weights = 8192 * synth.Q_LORA * 2 + 128 * synth.HIDDEN * 2 + 64 * synth.HIDDEN * 4
+        acts = T * (synth.HIDDEN * 2 + synth.Q_LORA * 2 + 8192 * 2 + 128 * 2 + 64 * 4)
+        info = {"bound": "tensor" if T >= 1024 else "hbm", "algorithmic_flops": flops,
+                "algorithmic_bytes": weights + acts, "kernel": "gemm_bf16_kernel (q, k, head weights)",
+                "config": {"tokens": T, "hidden": synth.HIDDEN, "q_lora": synth.Q_LORA}}
+    elif row == "mla":
+        B, H, T, k = 128, 128, 16384, 2048
+        q = torch.randn((B, H, 576), device=dev, generator=g).to(torch.bfloat16)
+        kv = torch.randn((B, T, 576), device=dev, generator=g).to(torch.bfloat16)
+        idx = torch.stack([torch.randperm(T, device=dev, generator=g)[:k] for _ in range(B)]).to(torch.int32)
+        out = torch.empty((B, H, 512), device=dev, dtype=torch.float32)
+        fn = lambda: X.sparse_mla_decode(q, kv, idx, 576 ** -0.5, out=out)
+        info = {"bound": "tensor", "algorithmic_flops": 2.0 * B * H * k * (576 + 512),
+                "algorithmic_bytes": B * k * 576 * 2 + B * H * (576 * 2 + 512 * 4),
+                "kernel": "sparse_mla_tc_kernel", "config": {"B": B, "H": H, "k": k, "T_cap": T}}
+    else:
+        raise SystemExit(f"--row: one of {', '.join(ROWS)}")
+    flush = l2_flush_buffer(torch, dev)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize(dev)
+    times = []
+    for _ in range(max(1, args.steps)):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize(dev)
+        times.append(a.elapsed_time(b) * 1e3)
+    us = statistics.median(times)
+    line = {"row": row, "us": us, "us_min": min(times), "steps": len(times), "warmup": args.warmup,
+            "status": list(X.status()), "l2": "flushed before each launch", "data": "synthetic", **info}
+    if "algorithmic_bytes" in info:
+        line["achieved_gbs"] = info["algorithmic_bytes"] / (us * 1e-6) / 1e9
+        line["frac_of_measured_hbm"] = line["achieved_gbs"] / hbm
+    if "algorithmic_flops" in info:
+        line["achieved_tflops"] = info["algorithmic_flops"] / (us * 1e-6) / 1e12
+        line["frac_of_measured_bf16"] = line["achieved_tflops"] / bf16
+    print(json.dumps(line))
+
+
 # ---------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -436,9 +552,17 @@ def main():
     ap.add_argument("--scale-storage", choices=["f32", "e8m0"], default="f32",
                     help="key scales as float32 (the workloads' layout) or one e8m0 byte per key "
                          "(ue8m0 workloads only)")
+    ap.add_argument("--row", choices=ROWS, default=None,
+                    help="time one widened row's launch alone (for its own numbers and ncu captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank, world, local_rank = env_rank()
+    if args.row is not None:
+        import torch
+        torch.cuda.set_device(local_rank)
+        hbm, bf16, _, _ = measured_peaks()
+        row_bench(args, torch.device("cuda", local_rank), hbm, bf16)
+        return
 
     if args.impl == "reference":
         if rank != 0:
@@ -500,7 +624,7 @@ def result_line(r, args, world, hbm, bf16, peak_src):
                 "frac_of_datasheet_fp8": achieved / DATASHEET_FP8_TFLOPS,
                 "kernel": "flat_score_kernel (tcgen05 FP8 scorer, fp32 scores to the workspace)",
                 "kernel_us": r["score_ms"] * 1e3, "algorithmic_flops": r["flops"],
-                "timing": "back-to-back launches between two CUDA events"}
+                "timing": "launches recorded back to back in a CUDA graph, one replay between two CUDA events"}
     else:
         achieved = r["score_bytes"] / score_s / 1e9
         traffic = (profile_traffic(PROFILE_SCORE, r["key_rows"])
@@ -513,7 +637,7 @@ def result_line(r, args, world, hbm, bf16, peak_src):
                 "kernel": "flat_score_kernel (tcgen05 FP8 scorer, fp32 scores to the workspace)" if r["two_pass"]
                 else "score_kernel (fused score + top-k)",
                 "kernel_us": r["score_ms"] * 1e3, "algorithmic_bytes": r["score_bytes"],
-                "timing": "back-to-back launches between two CUDA events"}
+                "timing": "launches recorded back to back in a CUDA graph, one replay between two CUDA events"}
     l2 = ("L2 flushed (a write of twice the L2 size) before each step, outside the timed events"
           if r["l2_flushed"] else
           "inputs larger than L2: %.0f MB FP8 cache streamed per step"
