@@ -58,6 +58,11 @@ int launch_flat_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cac
                       int scale_fmt, const int32_t* lengths, int B, int n, int T_cap, int max_len, int causal,
                       float* scores, int64_t ld, cudaStream_t stream);
 
+// Sparse latent attention on the tensor cores (mla_tc.cu): IDX_ERR_UNSUPPORTED
+// when the shape is not one it serves (H not a multiple of 128, q unaligned).
+int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, const int32_t* indices, int B, int H, int64_t T_cap,
+                         int k, float softmax_scale, float* out, cudaStream_t stream);
+
 struct DebugState {
   unsigned int flags;
   unsigned long long budget_ns;

@@ -10,7 +10,8 @@
 // so that 32 rows read at one column hit 32 banks), lane t of each warp scores
 // row t for its head, the warp updates its running max / sum (online softmax),
 // and each lane accumulates 16 of the head's 512 output columns.  Arithmetic is
-// fp32 on the CUDA cores.
+// fp32 on the CUDA cores.  This kernel serves head counts that are not a
+// multiple of 128; blocks of 128 heads run on the tensor cores (mla_tc.cu).
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -143,6 +144,10 @@ extern "C" int idx_sparse_mla_decode(const uint16_t* q, const uint16_t* kv, cons
   if (B == 0) return IDX_OK;
   if (!q || !kv || !indices || !out) return IDX_ERR_NULL;
   if (reinterpret_cast<uintptr_t>(kv) & 15) return IDX_ERR_ALIGN;
+  // 128-head blocks run on the tensor cores; other head counts on the CUDA cores
+  const int rt = launch_sparse_mla_tc(q, kv, indices, B, H, T_cap, k, softmax_scale, out,
+                                      reinterpret_cast<cudaStream_t>(stream));
+  if (rt != IDX_ERR_UNSUPPORTED) return rt;
   const int64_t blocks = static_cast<int64_t>(B) * (H / kMlaHeads);
   if (blocks > 0x7FFFFFFF) return IDX_ERR_SHAPE;
   const int smem = static_cast<int>(sizeof(MlaSmem));
