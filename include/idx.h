@@ -93,7 +93,7 @@ enum idx_status_code {
   IDX_ERR_DEVICE = -7,      /* idx_status: a kernel set the device error word */
   IDX_ERR_CUDA = -8,        /* idx_status: the stream itself reported a CUDA error */
   IDX_ERR_UNSUPPORTED = -9, /* no device code for this GPU (not sm_100) */
-  IDX_ERR_SCRATCH = -10     /* idx_score_topk_noalloc: the call needs more than the library's fixed scratch */
+  IDX_ERR_SCRATCH = -10     /* the scratch is too small: idx_score_topk_noalloc's fixed scratch, idx_project's ws */
 };
 
 /* Bits of the device error word (returned by idx_device_error_bits). */
@@ -192,20 +192,23 @@ IDX_API int idx_front_quant_append(const uint16_t* q_proj, const float* w_raw, c
  * idx_project — the three projections that open the Indexer.forward excerpt
  * ("Index scores" page): q = wq_b(qr) viewed as 64 heads of 128 features,
  * k = wk(x), and the head weights weights_proj(x.float()).
- *   x      [tokens, hidden] bf16 (hidden a multiple of 128), the hidden state.
+ *   x      [tokens, hidden] bf16 (hidden a multiple of 64), the hidden state.
  *   qr     [tokens, q_lora] bf16 (q_lora a multiple of 64), the low-rank query.
  *   wq_b   [64·128, q_lora] bf16, wk [128, hidden] bf16: Linear weights [out, in].
  *   w_proj [64, hidden] fp32.
  *   q_proj [tokens, 64, 128] bf16 out, k_proj [tokens, 128] bf16 out: the fp32
  *          products (tensor cores, fp32 accumulation) rounded to nearest-even bf16;
  *          ready for idx_front_quant_append.
- *   w_raw  [tokens, 64] fp32 out: Σ_k x·w_proj in fp32, k ascending (CUDA cores).
- *   ws / ws_bytes: scratch of idx_project_workspace_size(tokens, hidden, q_lora)
- *          bytes (16-byte aligned) for the fp32 partial sums of a product split
- *          over K when few tokens cannot fill the GPU; a smaller workspace (or
- *          none) means fewer splits, never an error.
- * All bf16 pointers and ws must be 16-byte aligned.  Errors: IDX_ERR_SHAPE,
- * IDX_ERR_NULL, IDX_ERR_ALIGN.
+ *   w_raw  [tokens, 64] fp32 out: Σ_k x·w_proj in fp32 on the tensor cores, with
+ *          w_proj split into three bf16 parts hi + mid + lo (equal to it within
+ *          2^-24 relative), each part's products summed in fp32, the three sums
+ *          added (lo + mid) + hi.
+ *   ws / ws_bytes: scratch of at least idx_project_workspace_size(tokens, hidden,
+ *          q_lora) bytes (16-byte aligned, required): the three bf16 parts of
+ *          w_proj (written every call) and the fp32 partial sums of products split
+ *          over K when few tokens cannot fill the GPU (added in a fixed order).
+ * All pointers except w_proj must be 16-byte aligned.  Errors: IDX_ERR_SHAPE,
+ * IDX_ERR_NULL (ws included), IDX_ERR_ALIGN, IDX_ERR_SCRATCH (ws_bytes too small).
  */
 IDX_API size_t idx_project_workspace_size(int64_t tokens, int hidden, int q_lora);
 IDX_API int idx_project(const uint16_t* x, const uint16_t* qr, int64_t tokens, int hidden, int q_lora,
@@ -335,8 +338,11 @@ IDX_API int idx_merge_topk(const idx_cand_t* cand, int G, int64_t rows, int kin,
  *   softmax_scale: finite; s = softmax_scale · q·kv.
  *   out [B, H, 512] fp32 (caller-owned): Σ_t softmax(s)_t · kv[t, 0:512]
  *          over the selected t; 0 for a row that selects nothing.
- * Arithmetic: fp32 on the CUDA cores (online softmax over chunks of 32
- * positions).  Errors: IDX_ERR_SHAPE (B < 0, H not a positive multiple of 16,
+ * Arithmetic: when H is a multiple of 128 (and q 16-byte aligned), on the
+ * tensor cores — bf16 products accumulated in fp32, the softmax weights
+ * rounded to bf16 for the weighted sum (their sum taken as rounded), chunks of
+ * 64 positions; otherwise fp32 on the CUDA cores (online softmax over chunks
+ * of 32 positions).  Errors: IDX_ERR_SHAPE (B < 0, H not a positive multiple of 16,
  * T_cap ≤ 0, a non-finite scale), IDX_ERR_K (k ≤ 0), IDX_ERR_NULL, IDX_ERR_ALIGN.
  */
 IDX_API int idx_sparse_mla_decode(const uint16_t* q, const uint16_t* kv, const int32_t* indices, int B, int H,

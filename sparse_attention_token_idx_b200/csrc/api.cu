@@ -231,7 +231,7 @@ extern "C" const char* idx_error_string(int code) {
     case IDX_ERR_DEVICE: return "a kernel reported an error (see idx_device_error_bits)";
     case IDX_ERR_CUDA: return "the stream reported a CUDA error";
     case IDX_ERR_UNSUPPORTED: return "no device code for this GPU (sm_100a required)";
-    case IDX_ERR_SCRATCH: return "the call needs more scratch than the library's fixed 64 MiB buffer";
+    case IDX_ERR_SCRATCH: return "the scratch is too small (the library's fixed 64 MiB buffer, or the caller's workspace)";
     default: return "unknown status";
   }
 }

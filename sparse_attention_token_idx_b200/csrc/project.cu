@@ -15,8 +15,12 @@
 // When M is small (decode: one token per sequence) the tile grid cannot fill
 // the GPU, so K is split over S CTAs that write fp32 partial sums; a second
 // kernel adds the S slices in a fixed order and rounds once to bf16.
-// The head weights are an fp32 product on the CUDA cores (x is bf16, the
-// weights fp32; each output is a sequential fp32 sum over k).
+// The head weights x·w_projᵀ (x bf16, w_proj fp32) run on the same tensor-core
+// GEMM: every fp32 weight is split into three bf16 parts, hi = bf16(w),
+// mid = bf16(w − hi), lo = bf16(w − hi − mid), which carry its 24 significand
+// bits, so x·w = x·hi + x·mid + x·lo with every product exact in fp32.  The
+// three parts are stacked as the 192 rows of one B operand; the epilogue adds
+// the three column groups per head, (lo + mid) + hi, in fp32.
 // Every wait is bounded; a CTA that gives up raises IDX_DEV_ERR_TIMEOUT,
 // waits for its copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -61,7 +65,7 @@ __device__ __forceinline__ uint32_t bf16_pair(float lo, float hi) {
 struct GemmParams {
   int M, N, K;
   int k_tiles;             // K tiles per CTA (its split-K slice)
-  void* out;               // bf16 [M, N] (S = 1) or fp32 partials [S, M, N]
+  void* out;               // bf16 [M, N] or fp32 partials [S, M, N]; GROUPS = 3: fp32 [M, N / 3] or [S, M, N / 3]
   int partial;             // write fp32 partials of this CTA's slice
   unsigned long long budget_ns;
   unsigned int* err;
@@ -75,11 +79,14 @@ struct GemmCfg {
   static constexpr int kOffBar = STAGES * kStage;
   static constexpr int kOffMisc = kOffBar + (2 * STAGES + 2) * 8;
   static constexpr int kSmem = 1024 + kOffMisc + 16;
-  static constexpr int kTmemCols = BN < 32 ? 32 : BN;
+  static constexpr int kTmemCols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;   // a power of two
 };
 
-// grid: x = N / BN column tiles, y = row tiles, z = split-K slices
-template <int BN, int STAGES>
+// grid: x = N / BN column tiles, y = row tiles, z = split-K slices.
+// GROUPS = 1: C tile to bf16 (or fp32 partials).  GROUPS = 3: the BN columns are
+// three stacked groups (weight parts hi, mid, lo); the output is their fp32 sum,
+// BN / 3 columns wide, as the result (one slice) or as slice partials.
+template <int BN, int STAGES, int GROUPS>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                      const GemmParams p) {
@@ -170,6 +177,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (ok) {
       tc_fence_after();
       const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+      if constexpr (GROUPS == 3) {
+        constexpr int kOut = BN / 3;
+        static_assert(kOut % 32 == 0, "column groups of whole TMEM loads");
+#pragma unroll 1
+        for (int c = 0; c < kOut / 32; ++c) {
+          float hi[32], mid[32], lo[32];
+          tmem_ld32(lane_base + static_cast<uint32_t>(c * 32), hi);
+          tmem_ld32(lane_base + static_cast<uint32_t>(kOut + c * 32), mid);
+          tmem_ld32(lane_base + static_cast<uint32_t>(2 * kOut + c * 32), lo);
+          if (row < p.M) {
+            float* dst = static_cast<float*>(p.out) + (static_cast<int64_t>(blockIdx.z) * p.M + row) * kOut + c * 32;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + i) =
+                  make_float4((lo[i] + mid[i]) + hi[i], (lo[i + 1] + mid[i + 1]) + hi[i + 1],
+                              (lo[i + 2] + mid[i + 2]) + hi[i + 2], (lo[i + 3] + mid[i + 3]) + hi[i + 3]);
+          }
+        }
+      } else {
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         float v[32];
@@ -194,6 +220,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+      }
     }
   }
   __syncthreads();
@@ -213,54 +240,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
-// out[m, n] = bf16(Σ_s part[s, m, n]), slices added in order s = 0, 1, …
-__global__ void splitk_reduce_kernel(const float* __restrict__ part, int S, int64_t MN,
-                                     __nv_bfloat16* __restrict__ out) {
+// out[i] = Σ_s part[s, i], slices added in order s = 0, 1, …, then rounded
+// once to the output type (bf16 to nearest-even, or kept fp32).
+template <typename OutT>
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int S, int64_t MN, OutT* __restrict__ out) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < MN;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     float acc = part[i];
     for (int s = 1; s < S; ++s) acc += part[s * MN + i];
-    out[i] = __float2bfloat16_rn(acc);
+    if constexpr (sizeof(OutT) == 2)
+      out[i] = __float2bfloat16_rn(acc);
+    else
+      out[i] = acc;
   }
 }
 
-// Head weights on the CUDA cores: w[t, h] = Σ_k fl32(x[t, k]) · W[h, k] in fp32,
-// k ascending.  A CTA takes 8 tokens × 64 heads; x and W chunks of 128 k are
-// staged in shared memory (W transposed, so that a warp reads 32 heads of one k).
-constexpr int kWTok = 8;
-constexpr int kWChunk = 128;
-
-__global__ void __launch_bounds__(256) head_weights_kernel(const uint16_t* __restrict__ x,
-                                                           const float* __restrict__ W, int64_t tokens, int hidden,
-                                                           float* __restrict__ w_out) {
-  __shared__ float xs[kWTok][kWChunk];
-  __shared__ float wt[kWChunk][IDX_HEADS + 1];
-  const int tid = threadIdx.x;
-  const int h = tid & 63;                  // head
-  const int tq = tid >> 6;                 // tokens tq and tq + 4
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kWTok;
-  float acc0 = 0.f, acc1 = 0.f;
-  for (int k0 = 0; k0 < hidden; k0 += kWChunk) {
-    __syncthreads();
-    for (int i = tid; i < kWTok * kWChunk; i += blockDim.x) {
-      const int tt = i / kWChunk, kk = i % kWChunk;
-      const int64_t t = t0 + tt;
-      xs[tt][kk] = t < tokens ? __uint_as_float(static_cast<uint32_t>(x[t * hidden + k0 + kk]) << 16) : 0.f;
-    }
-    for (int i = tid; i < IDX_HEADS * kWChunk; i += blockDim.x) {
-      const int hh = i / kWChunk, kk = i % kWChunk;
-      wt[kk][hh] = W[static_cast<int64_t>(hh) * hidden + k0 + kk];
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < kWChunk; ++kk) {
-      const float wv = wt[kk][h];
-      acc0 = fmaf(xs[tq][kk], wv, acc0);
-      acc1 = fmaf(xs[tq + 4][kk], wv, acc1);
-    }
+// w_proj [64, hidden] fp32 → three bf16 parts [3][64][hidden]: hi = bf16(w),
+// mid = bf16(w − hi), lo = bf16(w − hi − mid).  Both differences are exact in
+// fp32 (each subtracts a rounding of the value itself, Sterbenz), and the last
+// rounding is of a remainder below 2⁻¹⁶·|w|, so hi + mid + lo = w within 2⁻²⁴·|w|.
+__global__ void split_weights_kernel(const float* __restrict__ w, int64_t count, __nv_bfloat16* __restrict__ parts) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float v = w[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);
+    parts[i] = hi;
+    parts[count + i] = mid;
+    parts[2 * count + i] = __float2bfloat16_rn(r2);
   }
-  if (t0 + tq < tokens) w_out[(t0 + tq) * IDX_HEADS + h] = acc0;
-  if (t0 + tq + 4 < tokens) w_out[(t0 + tq + 4) * IDX_HEADS + h] = acc1;
+}
+
+int grid_for(int64_t count) {
+  const int64_t b = (count + 255) / 256;
+  return static_cast<int>(b < 148 * 8 ? b : 148 * 8);
 }
 
 // Split of K for an M × N product: enough CTAs to cover the SMs, slices of at
@@ -288,8 +303,8 @@ size_t partial_floats(int64_t M, int N, int K, int sms) {
   return S > 1 ? static_cast<size_t>(S) * static_cast<size_t>(M) * static_cast<size_t>(N) : 0;
 }
 
-template <int BN>
-int launch_gemm(const uint16_t* A, const uint16_t* Bw, int64_t M, int N, int K, uint16_t* out, float* part, int S,
+template <int BN, int GROUPS>
+int launch_gemm(const uint16_t* A, const uint16_t* Bw, int64_t M, int N, int K, void* out, float* part, int S,
                 int per, cudaStream_t stream) {
   constexpr int STAGES = 4;
   using C = GemmCfg<BN, STAGES>;
@@ -297,7 +312,7 @@ int launch_gemm(const uint16_t* A, const uint16_t* Bw, int64_t M, int N, int K, 
   if (!make_tmap_2d_bf16_sw128(&ta, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M), kGemmM))
     return IDX_ERR_ALIGN;
   if (!make_tmap_2d_bf16_sw128(&tb, Bw, static_cast<uint64_t>(K), static_cast<uint64_t>(N), BN)) return IDX_ERR_ALIGN;
-  auto kern = gemm_bf16_kernel<BN, STAGES>;
+  auto kern = gemm_bf16_kernel<BN, STAGES, GROUPS>;
   if (const int r = ensure_smem_limit(reinterpret_cast<const void*>(kern), C::kSmem)) return r;
   GemmParams p;
   p.M = static_cast<int>(M);
@@ -305,7 +320,7 @@ int launch_gemm(const uint16_t* A, const uint16_t* Bw, int64_t M, int N, int K, 
   p.K = K;
   p.k_tiles = per;
   p.partial = S > 1 ? 1 : 0;
-  p.out = S > 1 ? static_cast<void*>(part) : static_cast<void*>(out);
+  p.out = S > 1 ? static_cast<void*>(part) : out;
   const DebugState dbg = debug_state();
   p.budget_ns = dbg.budget_ns;
   p.err = device_error_word();
@@ -315,24 +330,22 @@ int launch_gemm(const uint16_t* A, const uint16_t* Bw, int64_t M, int N, int K, 
   kern<<<grid, kGemmThreads, C::kSmem, stream>>>(ta, tb, p);
   if (const int r = check_launch()) return r;
   if (S > 1) {
-    const int64_t MN = M * N;
-    const int blocks = static_cast<int>((MN + 255) / 256 < 148 * 8 ? (MN + 255) / 256 : 148 * 8);
-    splitk_reduce_kernel<<<blocks, 256, 0, stream>>>(part, S, MN, reinterpret_cast<__nv_bfloat16*>(out));
+    const int64_t MN = M * (N / GROUPS);
+    if constexpr (GROUPS == 1)
+      splitk_reduce_kernel<<<grid_for(MN), 256, 0, stream>>>(part, S, MN, static_cast<__nv_bfloat16*>(out));
+    else
+      splitk_reduce_kernel<<<grid_for(MN), 256, 0, stream>>>(part, S, MN, static_cast<float*>(out));
     return check_launch();
   }
   return IDX_OK;
 }
 
-// One bf16 projection: the column tile and the split-K slices for this shape
-// (fewer slices when the workspace is smaller than the partial sums need).
-int project_bf16(const uint16_t* A, const uint16_t* Bw, int64_t M, int N, int K, uint16_t* out, float* ws,
-                 size_t ws_floats, cudaStream_t stream) {
-  const int sms = num_sms();
-  const int BN = column_tile(M, N, sms);
+// The split-K slices of one product: as split_k proposes, then fewer while the
+// partial sums (M × out_cols fp32 per slice) would not fit in part_floats.
+void slices_for(int64_t M, int N, int BN, int out_cols, int K, size_t part_floats, int& S, int& per) {
   const int k_tiles = K / kGemmK;
-  int S, per;
-  split_k(((M + kGemmM - 1) / kGemmM) * (N / BN), k_tiles, sms, S, per);
-  while (S > 1 && static_cast<size_t>(S) * static_cast<size_t>(M) * N > ws_floats) {
+  split_k(((M + kGemmM - 1) / kGemmM) * (N / BN), k_tiles, num_sms(), S, per);
+  while (S > 1 && static_cast<size_t>(S) * static_cast<size_t>(M) * out_cols > part_floats) {
     per *= 2;
     S = (k_tiles + per - 1) / per;
   }
@@ -340,11 +353,26 @@ int project_bf16(const uint16_t* A, const uint16_t* Bw, int64_t M, int N, int K,
     S = 1;
     per = k_tiles;
   }
+}
+
+// One bf16 projection: the column tile and the split-K slices for this shape.
+int project_bf16(const uint16_t* A, const uint16_t* Bw, int64_t M, int N, int K, uint16_t* out, float* part,
+                 size_t part_floats, cudaStream_t stream) {
+  const int BN = column_tile(M, N, num_sms());
+  int S, per;
+  slices_for(M, N, BN, N, K, part_floats, S, per);
   switch (BN) {
-    case 256: return launch_gemm<256>(A, Bw, M, N, K, out, ws, S, per, stream);
-    case 128: return launch_gemm<128>(A, Bw, M, N, K, out, ws, S, per, stream);
-    default: return launch_gemm<64>(A, Bw, M, N, K, out, ws, S, per, stream);
+    case 256: return launch_gemm<256, 1>(A, Bw, M, N, K, out, part, S, per, stream);
+    case 128: return launch_gemm<128, 1>(A, Bw, M, N, K, out, part, S, per, stream);
+    default: return launch_gemm<64, 1>(A, Bw, M, N, K, out, part, S, per, stream);
   }
+}
+
+constexpr int kHeadCols = 3 * IDX_HEADS;   // the stacked weight parts: one 192-column tile
+
+// Bytes of the three bf16 weight parts, rounded up to keep what follows aligned.
+size_t weight_parts_bytes(int hidden) {
+  return (static_cast<size_t>(kHeadCols) * static_cast<size_t>(hidden) * 2 + 255) & ~static_cast<size_t>(255);
 }
 
 }  // namespace
@@ -353,34 +381,45 @@ int project_bf16(const uint16_t* A, const uint16_t* Bw, int64_t M, int N, int K,
 using namespace idx;
 
 extern "C" size_t idx_project_workspace_size(int64_t tokens, int hidden, int q_lora) {
-  if (tokens <= 0 || hidden <= 0 || q_lora <= 0 || hidden % 128 || q_lora % kGemmK) return 0;
+  if (tokens <= 0 || hidden <= 0 || q_lora <= 0 || hidden % kGemmK || q_lora % kGemmK) return 0;
   const int sms = num_sms();
   const size_t q = partial_floats(tokens, IDX_HEADS * IDX_DIM, q_lora, sms);
   const size_t k = partial_floats(tokens, IDX_DIM, hidden, sms);
-  return (q > k ? q : k) * sizeof(float);
+  int S, per;
+  split_k((tokens + kGemmM - 1) / kGemmM, hidden / kGemmK, sms, S, per);
+  const size_t w = S > 1 ? static_cast<size_t>(S) * static_cast<size_t>(tokens) * IDX_HEADS : 0;
+  size_t m = q > k ? q : k;
+  m = m > w ? m : w;
+  return weight_parts_bytes(hidden) + m * sizeof(float);
 }
 
 extern "C" int idx_project(const uint16_t* x, const uint16_t* qr, int64_t tokens, int hidden, int q_lora,
                            const uint16_t* wq_b, const uint16_t* wk, const float* w_proj, uint16_t* q_proj,
                            uint16_t* k_proj, float* w_raw, void* ws, size_t ws_bytes, idx_stream_t stream) {
   if (tokens < 0 || hidden <= 0 || q_lora <= 0) return IDX_ERR_SHAPE;
-  if (hidden % kWChunk || q_lora % kGemmK) return IDX_ERR_SHAPE;
+  if (hidden % kGemmK || q_lora % kGemmK) return IDX_ERR_SHAPE;
   if (tokens == 0) return IDX_OK;
-  if (!x || !qr || !wq_b || !wk || !w_proj || !q_proj || !k_proj || !w_raw) return IDX_ERR_NULL;
+  if (!x || !qr || !wq_b || !wk || !w_proj || !q_proj || !k_proj || !w_raw || !ws) return IDX_ERR_NULL;
   if (tokens > 0x7FFFFFFF / IDX_HEADS / IDX_DIM) return IDX_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(qr) | reinterpret_cast<uintptr_t>(wq_b) |
        reinterpret_cast<uintptr_t>(wk) | reinterpret_cast<uintptr_t>(q_proj) | reinterpret_cast<uintptr_t>(k_proj) |
-       reinterpret_cast<uintptr_t>(ws)) & 15)
+       reinterpret_cast<uintptr_t>(w_raw) | reinterpret_cast<uintptr_t>(ws)) & 15)
     return IDX_ERR_ALIGN;
+  const size_t parts_bytes = weight_parts_bytes(hidden);
+  if (ws_bytes < idx_project_workspace_size(tokens, hidden, q_lora)) return IDX_ERR_SCRATCH;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  float* part = static_cast<float*>(ws);
-  const size_t part_floats = ws ? ws_bytes / sizeof(float) : 0;
-  int r = project_bf16(qr, wq_b, tokens, IDX_HEADS * IDX_DIM, q_lora, q_proj, part, part_floats, s);
+  uint16_t* parts = static_cast<uint16_t*>(ws);
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + parts_bytes);
+  const size_t part_floats = (ws_bytes - parts_bytes) / sizeof(float);
+  const int64_t wcount = static_cast<int64_t>(IDX_HEADS) * hidden;
+  split_weights_kernel<<<grid_for(wcount), 256, 0, s>>>(w_proj, wcount, reinterpret_cast<__nv_bfloat16*>(parts));
+  int r = check_launch();
+  if (r != IDX_OK) return r;
+  r = project_bf16(qr, wq_b, tokens, IDX_HEADS * IDX_DIM, q_lora, q_proj, part, part_floats, s);
   if (r != IDX_OK) return r;
   r = project_bf16(x, wk, tokens, IDX_DIM, hidden, k_proj, part, part_floats, s);
   if (r != IDX_OK) return r;
-  const int64_t blocks = (tokens + kWTok - 1) / kWTok;
-  if (blocks > 0x7FFFFFFF) return IDX_ERR_SHAPE;
-  head_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, w_proj, tokens, hidden, w_raw);
-  return check_launch();
+  int S, per;
+  slices_for(tokens, kHeadCols, kHeadCols, IDX_HEADS, hidden, part_floats, S, per);
+  return launch_gemm<kHeadCols, 3>(x, parts, tokens, kHeadCols, hidden, w_raw, part, S, per, s);
 }
