@@ -47,6 +47,7 @@ ROWS = [
     ("large-k", 64, 16384, 16384, 4096, "random"),     # positions written without staging
     ("ragged", 80, 16381, 16384, 512, "random"),       # lengths not multiples of 4 (ld is)
     ("unaligned-ld", 70, 3001, 3001, 700, "random"),   # ld % 4 != 0: cluster kernel
+    ("sample-blind", 64, 16384, 16384, 2048, "strided"),  # the sampled positions all score low: radix fallback
 ]
 
 
@@ -61,6 +62,8 @@ def test_topk_many_rows(name, rows, L, ld, k, order):
         sc = sc - np.float32(0.01) * np.arange(ld, dtype=np.float32)
     elif order == "asc":
         sc = sc + np.float32(0.01) * np.arange(ld, dtype=np.float32)
+    elif order == "strided":
+        sc[:, :, ::4] -= np.float32(100.0)
     lengths = rng.integers(max(1, L - 700), L + 1, rows).astype(np.int32)
     lengths[0] = L
     lengths[1] = min(L, k)                       # every visible key selected
@@ -116,3 +119,27 @@ def test_fused_topk_matches_oracle_and_unfused(name, B, n, positions, T_cap, cau
             check_topk_row(idx[b, i], S[b, i], E[b, i], vis, k)
             # the fused kernel selects from the very fp32 scores idx_score writes
             check_topk_exact_row(idx[b, i], sc[b, i], vis, k)
+
+
+@pytest.mark.parametrize("zeroed", ["all", "sampled-positions"])
+def test_fused_topk_when_the_sample_cannot_place_the_threshold(zeroed):
+    """The one-CTA decode selection first estimates the threshold from a strided
+    sample of the row; when the sample has no spread (every sampled key scores
+    0) it hands the row to the exact radix selection.  Keys zeroed at every
+    position (all scores tie) or only at the sampled positions (every 4th of
+    16 384) must still give an exact top-k."""
+    from sparse_attention_token_idx_b200 import binding as X
+    B, T_cap, k = 4, 16384, 2048
+    case = synth.make_case("zeroed-" + zeroed, 77, B, 1, [T_cap - 1] * B, T_cap=T_cap, causal=False, fmt=1, k=k)
+    if zeroed == "all":
+        case.k_prior[:] = 0
+        case.k_new[:] = 0
+    else:
+        case.k_prior[:, ::4] = 0
+    kc, ks, lengths = gpu_state(case)
+    qc, w = gpu_queries(case)
+    idx = X.score_topk(qc, w, kc, ks, lengths, False, k, T_cap).cpu().numpy()
+    sc = X.score(qc, w, kc, ks, lengths, False, T_cap, ld=T_cap).cpu().numpy()
+    assert X.status() == (0, 0)
+    for b in range(B):
+        check_topk_exact_row(idx[b, 0], sc[b, 0], T_cap, k)
