@@ -5,20 +5,26 @@
 //
 // One CTA per (sequence, block of 128 heads, half of the 512 output columns):
 // the two halves recompute the same scores (a softmax needs all of them) and
-// each accumulates 256 output columns, so that the output accumulator
-// (128 lanes × 256 fp32 columns) and two score tiles fit TMEM together.
+// each accumulates 256 output columns.  The queries stay resident for the
+// whole walk: features 0-383 in TMEM as the A operand of the score MMAs (six
+// 64-feature tiles, two bf16 per 32-bit column), features 384-575 in shared
+// memory (three 128-byte-swizzled tiles, by TMA).  TMEM: query tiles at
+// columns 0-191, one 64-column score tile at 192, the output half at 256.
 // The selection is walked in chunks of 64 positions:
-//   warps 6-9   gather the chunk's rows (16-byte cp.async, 1152 B per row) into
+//   warps 6…    gather the chunk's rows (16-byte cp.async, 1152 B per row) into
 //               shared memory as nine 64-feature K tiles in the 128-byte swizzle
-//               layout (row = position); unselected slots are zeros;
-//   warp 0      streams the 128 heads' query tiles (nine 64-feature tiles of
-//               128 × 128 B) by TMA into a 3-stage ring, once per chunk;
+//               layout (row = position); unselected slots are zeros; two chunk
+//               buffers;
+//   warp 0      loads the three shared-memory query tiles once;
 //   warp 1      owns TMEM and issues tcgen05.mma kind::f16 (bf16 → fp32):
-//               S = Q · Kᵀ into one of two 64-column score tiles (N = 64,
-//               K = 576), and O += P · V (N = 256, K = 64 positions) where V is
-//               this CTA's four 64-feature tiles of the same gathered bytes read
-//               as an MN-major operand;
-//   warps 2-5   softmax, thread ↔ head: read the score row from TMEM, mask
+//               S = Q · Kᵀ into the score tile (N = 64, K = 576: 24 MMAs with
+//               A in TMEM, 12 with A in shared memory), and O += P · V (N = 256,
+//               K = 64 positions) where V is this CTA's four 64-feature tiles of
+//               the same gathered bytes read as an MN-major operand; the
+//               product of chunk c − 1 goes before the scores of chunk c, so
+//               that its buffer is refilled while those scores run;
+//   warps 2-5   load their head's query features 0-383 into TMEM at the start;
+//               then softmax, thread ↔ head: read the score row from TMEM, mask
 //               unselected slots, keep a running reference maximum m (raised
 //               only when a chunk's maximum exceeds it by more than 8, then the
 //               O row and the running sum are rescaled), p = exp(s − m) rounded
@@ -42,11 +48,13 @@ constexpr int kTcDim = 576;                // latent + rotary
 constexpr int kTcHalf = 256;               // output columns per CTA
 constexpr int kTcChunk = 64;               // positions per chunk
 constexpr int kTcKTiles = kTcDim / 64;     // 9 feature tiles of 64
-constexpr int kTcQStages = 3;
-constexpr int kTcThreads = 320;
-constexpr int kTcGatherThreads = 128;      // warps 6-9
-constexpr int kTcPieces = kTcChunk * (kTcDim / 8);   // 16-byte pieces of one chunk (4608)
+constexpr int kTcGatherWarps = 4;          // warps 6 … 6 + kTcGatherWarps − 1
+constexpr int kTcThreads = (6 + kTcGatherWarps) * 32;
+constexpr int kTcGatherThreads = kTcGatherWarps * 32;
+constexpr int kTcRowsPerWarp = 64 / kTcGatherWarps;   // chunk rows each gather warp copies
 constexpr float kTcRescale = 8.f;          // raise the reference maximum past this margin
+constexpr int kTcQTmemTiles = 6;           // query feature tiles held in TMEM (features 0-383)
+constexpr int kTcQSmemTiles = kTcKTiles - kTcQTmemTiles;   // the rest in shared memory
 
 constexpr int kQTile = kTcHeads * 128;               // 16 KB
 constexpr int kKvTile = kTcChunk * 128;              // 8 KB per 64-feature tile of a chunk
@@ -54,17 +62,19 @@ constexpr int kKvChunk = kTcKTiles * kKvTile;        // 72 KB
 constexpr int kPTile = kTcHeads * 128;               // 16 KB: 128 heads × 64 positions bf16
 
 constexpr int kOffQ = 0;
-constexpr int kOffKv = kOffQ + kTcQStages * kQTile;
+constexpr int kOffKv = kOffQ + kTcQSmemTiles * kQTile;
 constexpr int kOffP = kOffKv + 2 * kKvChunk;
 constexpr int kOffBar = kOffP + kPTile;
-// barriers: q_full[3] q_empty[3] kv_full[2] kv_empty[2] s_full[2] s_empty[2] p_full p_empty o_done drain
-constexpr int kNumBars = 3 + 3 + 2 + 2 + 2 + 2 + 4;
+// barriers: q_full kv_full[2] kv_empty[2] s_full s_empty p_full p_empty o_done drain
+constexpr int kNumBars = 1 + 2 + 2 + 6;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kTcSmem = 1024 + kOffMisc + 16;
 
-// TMEM columns: score tiles at 0 and 64, the output half at 256
-constexpr uint32_t kColS = 0;
+// TMEM columns: query tiles (32 columns each), the score tile, the output half
+constexpr uint32_t kColQ = 0;
+constexpr uint32_t kColS = kTcQTmemTiles * 32;
 constexpr uint32_t kColO = 256;
+static_assert(kColS + kTcChunk <= kColO, "TMEM columns");
 
 // kind::f16, A = B = bf16, D = f32; b_mn: B operand MN-major
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn) {
@@ -79,6 +89,17 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The same with A read from TMEM (row m in lane m, two bf16 per 32-bit column).
+__device__ __forceinline__ void mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -124,6 +145,7 @@ __device__ __forceinline__ uint32_t sw128(int r, int c) {
 }
 
 struct TcParams {
+  const uint16_t* q;         // [B, H, 576]
   const uint16_t* kv;        // [B, T_cap, 576]
   const int32_t* indices;    // [B, k]
   float* out;                // [B, H, 512]
@@ -142,16 +164,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* kv_s = smem + kOffKv;
   uint8_t* p_s = smem + kOffP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* q_full = bars;
-  uint64_t* q_empty = bars + 3;
-  uint64_t* kv_full = bars + 6;
-  uint64_t* kv_empty = bars + 8;
-  uint64_t* s_full = bars + 10;
-  uint64_t* s_empty = bars + 12;
-  uint64_t* p_full = bars + 14;
-  uint64_t* p_empty = bars + 15;
-  uint64_t* o_done = bars + 16;
-  uint64_t* drain_bar = bars + 17;
+  uint64_t* q_full = bars;          // the shared-memory query tiles have landed
+  uint64_t* kv_full = bars + 1;     // [2]
+  uint64_t* kv_empty = bars + 3;    // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* s_empty = bars + 6;
+  uint64_t* p_full = bars + 7;
+  uint64_t* p_empty = bars + 8;
+  uint64_t* o_done = bars + 9;
+  uint64_t* drain_bar = bars + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
@@ -165,16 +186,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint64_t budget = p.budget_ns;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 3; ++i) {
-      mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1);
-    }
+    mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kv_full[i], kTcGatherThreads);
       mbar_init(&kv_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 4);
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, 4);
     mbar_init(p_full, 4);
     mbar_init(p_empty, 1);
     mbar_init(o_done, 1);
@@ -182,65 +200,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmap_q);
+    // query features 384-575: three 64-feature tiles, once
+    mbar_arrive_expect_tx(q_full, kTcQSmemTiles * kQTile);
+    for (int t = 0; t < kTcQSmemTiles; ++t)
+      tma_load_2d(q_s + t * kQTile, &tmap_q, q_full, (kTcQTmemTiles + t) * 64, static_cast<int>(b * p.H + h0));
   }
   if (warp == 1) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  int q_issued = 0;
+  if (warp >= 2 && warp < 6) {
+    // query features 0-383 of head h into TMEM lane h: 32 columns per 64 features
+    const int h = (warp & 3) * 32 + lane;
+    const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (b * p.H + h0 + h) * kTcDim);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+#pragma unroll 1
+    for (int t = 0; t < kTcQTmemTiles; ++t) {
+      uint32_t r[32];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint4 v = __ldg(qrow + t * 8 + i);
+        r[4 * i] = v.x;
+        r[4 * i + 1] = v.y;
+        r[4 * i + 2] = v.z;
+        r[4 * i + 3] = v.w;
+      }
+      tmem_st32(lane_base + kColQ + static_cast<uint32_t>(t * 32), r);
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
   bool mma_issued = false;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ query tiles
-    if (lane == 0) {
-      const int total = nch * kTcKTiles;
-      for (int i = 0; i < total; ++i) {
-        const int s = i % kTcQStages;
-        if (i >= kTcQStages && !mbar_wait(&q_empty[s], ((i / kTcQStages) - 1) & 1, budget, abort_flag, p.err)) break;
-        mbar_arrive_expect_tx(&q_full[s], kQTile);
-        tma_load_2d(q_s + s * kQTile, &tmap_q, &q_full[s], (i % kTcKTiles) * 64,
-                    static_cast<int>(b * p.H + h0));
-        q_issued = i + 1;
-      }
-    }
-    __syncwarp();
+    // the query tiles were requested during set-up
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16(kTcHeads, kTcChunk, false);
       constexpr uint32_t id_o = idesc_bf16(kTcHeads, kTcHalf, true);
-      int qi = 0;
-      bool ok = true;
-      // S(c) for c = 0, 1, … and O += P(c) · V(c) one chunk behind, so that the
-      // softmax of chunk c overlaps the scores of chunk c + 1
+      bool ok = mbar_wait(q_full, 0, budget, abort_flag, p.err);
+      const uint32_t d_s = tmem + kColS;
+      // O += P(c − 1) · V(c − 1), then S(c): the product frees chunk c − 1's
+      // buffer before the scores of chunk c start, so that the gather of chunk
+      // c + 1 runs under the MMAs of chunk c (the scores are issued as soon as
+      // the softmax has read the previous ones out of TMEM)
       for (int c = 0; c <= nch && ok; ++c) {
-        if (c < nch) {
-          const int buf = c & 1;
-          ok = mbar_wait(&kv_full[buf], (c >> 1) & 1, budget, abort_flag, p.err);
-          if (ok && c >= 2) ok = mbar_wait(&s_empty[buf], ((c >> 1) - 1) & 1, budget, abort_flag, p.err);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t kv_addr = smem_u32(kv_s + buf * kKvChunk);
-          const uint32_t d = tmem + kColS + static_cast<uint32_t>(buf * kTcChunk);
-          for (int kt = 0; kt < kTcKTiles; ++kt, ++qi) {
-            const int s = qi % kTcQStages;
-            if (!mbar_wait(&q_full[s], (qi / kTcQStages) & 1, budget, abort_flag, p.err)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t q_addr = smem_u32(q_s + s * kQTile);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)   // 16 bf16 (32 bytes) per instruction
-              mma_f16(d, smem_desc_k128_sw128(q_addr + kk * 32),
-                      smem_desc_k128_sw128(kv_addr + kt * kKvTile + kk * 32), id_s, (kt > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&q_empty[s]);
-            mma_issued = true;
-          }
-          if (!ok) break;
-          mma_commit(&s_full[buf]);
-        }
         if (c >= 1) {
           const int pc = c - 1, buf = pc & 1;
           if (!mbar_wait(p_full, pc & 1, budget, abort_flag, p.err)) break;
@@ -257,6 +265,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (pc == nch - 1) mma_commit(o_done);
           mma_issued = true;
         }
+        if (c < nch) {
+          const int buf = c & 1;
+          ok = mbar_wait(&kv_full[buf], (c >> 1) & 1, budget, abort_flag, p.err);
+          if (ok && c >= 1) ok = mbar_wait(s_empty, (c - 1) & 1, budget, abort_flag, p.err);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t kv_addr = smem_u32(kv_s + buf * kKvChunk);
+          for (int kt = 0; kt < kTcKTiles; ++kt) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {   // 16 bf16 (32 bytes) per instruction
+              const uint64_t bd = smem_desc_k128_sw128(kv_addr + kt * kKvTile + kk * 32);
+              const uint32_t acc = (kt > 0 || kk > 0) ? 1u : 0u;
+              if (kt < kTcQTmemTiles)
+                mma_f16_ta(d_s, tmem + kColQ + static_cast<uint32_t>(kt * 32 + kk * 8), bd, id_s, acc);
+              else
+                mma_f16(d_s, smem_desc_k128_sw128(smem_u32(q_s + (kt - kTcQTmemTiles) * kQTile) + kk * 32), bd, id_s,
+                        acc);
+            }
+          }
+          mma_commit(s_full);
+          mma_issued = true;
+        }
       }
       if (mma_issued) mma_commit(drain_bar);
     }
@@ -270,24 +300,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int c = 0; c < nch && ok; ++c) {
-      const int buf = c & 1;
-      int w = 1;
-      if (lane == 0) w = mbar_wait(&s_full[buf], (c >> 1) & 1, budget, abort_flag, p.err) ? 1 : 0;
-      if (!__shfl_sync(0xFFFFFFFFu, w, 0)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t r[64];
-      tmem_ld32_nowait(lane_base + kColS + static_cast<uint32_t>(buf * kTcChunk), r);
-      tmem_ld32_nowait(lane_base + kColS + static_cast<uint32_t>(buf * kTcChunk + 32), r + 32);
-      tmem_wait();
-      tmem_regs_ready(r);
-      tmem_regs_ready(r + 32);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[buf]);
-      // which of the chunk's 64 slots select a cache row: two indices per lane
+      // which of the chunk's 64 slots select a cache row (two indices per lane),
+      // read before the wait for the scores so that the loads overlap it
       uint32_t vmask[2];
 #pragma unroll
       for (int g = 0; g < 2; ++g) {
@@ -295,6 +309,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int t = j < p.k ? __ldg(sel + j) : -1;
         vmask[g] = __ballot_sync(0xFFFFFFFFu, t >= 0 && t < p.T_cap);
       }
+      int w = 1;
+      if (lane == 0) w = mbar_wait(s_full, c & 1, budget, abort_flag, p.err) ? 1 : 0;
+      if (!__shfl_sync(0xFFFFFFFFu, w, 0)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[64];
+      tmem_ld32_nowait(lane_base + kColS, r);
+      tmem_ld32_nowait(lane_base + kColS + 32u, r + 32);
+      tmem_wait();
+      tmem_regs_ready(r);
+      tmem_regs_ready(r + 32);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_empty);
       float cmax = -INFINITY;
 #pragma unroll
       for (int j = 0; j < 64; ++j) {
@@ -377,14 +407,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ gather
-    const int gt = threadIdx.x - 6 * 32;              // 0 … 127
+    // gather warp gw copies rows gw, gw + W, gw + 2W, … of a chunk (W gather
+    // warps): its first lanes fetch those rows' positions once, then each row
+    // goes out as 72 consecutive 16-byte pieces across the warp (lane l:
+    // pieces l, l + 32, l + 64)
+    const int gw = warp - 6;
     const uint16_t* kvb = p.kv + b * p.T_cap * kTcDim;
     const int32_t* sel = p.indices + b * p.k;
     bool ok = true;
     for (int c = 0; c <= nch && ok; ++c) {
       // the previous chunk's copies have landed: make them visible to the MMAs
       // and announce them first — the buffer this chunk needs is freed by the
-      // product of chunk c − 2, which the MMA warp issues after the scores of
+      // product of chunk c − 2, which the MMA warp issues before the scores of
       // chunk c − 1
       if (c >= 1) {
         cp_async_wait<0>();
@@ -393,23 +427,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (c == nch) break;
       const int buf = c & 1;
+      int pos = -1;
+      if (lane < kTcRowsPerWarp) {
+        const int j = c * kTcChunk + gw + kTcGatherWarps * lane;
+        pos = j < p.k ? __ldg(sel + j) : -1;
+      }
       if (c >= 2) {
         int w = 1;
-        if ((gt & 31) == 0) w = mbar_wait(&kv_empty[buf], ((c >> 1) - 1) & 1, budget, abort_flag, p.err) ? 1 : 0;
+        if (lane == 0) w = mbar_wait(&kv_empty[buf], ((c >> 1) - 1) & 1, budget, abort_flag, p.err) ? 1 : 0;
         if (!__shfl_sync(0xFFFFFFFFu, w, 0)) {
           ok = false;
           break;
         }
       }
       const uint32_t base = smem_u32(kv_s + buf * kKvChunk);
-      for (int i = gt; i < kTcPieces; i += kTcGatherThreads) {
-        const int r = i / (kTcDim / 8), piece = i - r * (kTcDim / 8);
-        const int kt = piece >> 3, c16 = piece & 7;
-        const int j = c * kTcChunk + r;
-        const int t = j < p.k ? __ldg(sel + j) : -1;
-        const uint32_t dst = base + static_cast<uint32_t>(kt * kKvTile) + sw128(r, c16);
-        if (t >= 0 && t < p.T_cap) cp_async16(dst, kvb + static_cast<int64_t>(t) * kTcDim + piece * 8);
-        else asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+#pragma unroll 1
+      for (int i = 0; i < kTcRowsPerWarp; ++i) {
+        const int r = gw + kTcGatherWarps * i;
+        const int t = __shfl_sync(0xFFFFFFFFu, pos, i);
+        const bool valid = t >= 0 && t < p.T_cap;
+        const uint16_t* src = kvb + static_cast<int64_t>(valid ? t : 0) * kTcDim;
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+          const int piece = lane + 32 * q;
+          if (piece < kTcDim / 8) {
+            const uint32_t dst = base + static_cast<uint32_t>((piece >> 3) * kKvTile) + sw128(r, piece & 7);
+            if (valid) cp_async16(dst, src + piece * 8);
+            else asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+          }
+        }
       }
       cp_async_commit();
     }
@@ -419,8 +465,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // ------------------------------------------------------------ teardown
   if (warp == 0 && lane == 0) {
     int dummy = 0;
-    for (int i = q_issued > kTcQStages ? q_issued - kTcQStages : 0; i < q_issued; ++i)
-      mbar_wait(&q_full[i % kTcQStages], (i / kTcQStages) & 1, budget, &dummy, p.err);
+    mbar_wait(q_full, 0, budget, &dummy, p.err);   // the query tiles have landed before the memory goes
   }
   if (warp == 1 && lane == 0 && mma_issued) {
     int dummy = 0;
@@ -445,6 +490,7 @@ int launch_sparse_mla_tc(const uint16_t* q, const uint16_t* kv, const int32_t* i
   if (blocks > 0x7FFFFFFF) return IDX_ERR_SHAPE;
   if (const int r = ensure_smem_limit(reinterpret_cast<const void*>(sparse_mla_tc_kernel), kTcSmem)) return r;
   TcParams p;
+  p.q = q;
   p.kv = kv;
   p.indices = indices;
   p.out = out;
