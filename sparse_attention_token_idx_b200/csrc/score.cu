@@ -256,8 +256,8 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
       for (; t < ntiles; ++t) {
         const int s = t % STAGES;
         const int c = t % C::kScaleSlots;
-        if (!mbar_wait(&empty[s], ((t / STAGES) & 1) ^ 1, budget, abort_flag, p.err)) break;
-        if (!mbar_wait(&sc_empty[c], ((t / C::kScaleSlots) & 1) ^ 1, budget, abort_flag, p.err)) break;
+        if (!mbar_wait_sleep(&empty[s], ((t / STAGES) & 1) ^ 1, budget, abort_flag, p.err)) break;
+        if (!mbar_wait_sleep(&sc_empty[c], ((t / C::kScaleSlots) & 1) ^ 1, budget, abort_flag, p.err)) break;
         mbar_arrive_expect_tx(&full[s], kTileBytes + kTileKeys * (p.scale_u8 ? 1 : 4));
         const int tt = tile_of(t);
         tma_load_3d(k_s + s * kTileBytes, &tmap_k, &full[s], 0, start + tt * kTileKeys, b);
@@ -270,14 +270,14 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       if (p.debug_flags & 1u) mbar_wait(never_bar, 0, budget, abort_flag, p.err);  // fault injection: nothing arrives
-      if (ntiles > 0 && mbar_wait(q_full, 0, budget, abort_flag, p.err)) {
+      if (ntiles > 0 && mbar_wait_sleep(q_full, 0, budget, abort_flag, p.err)) {
         constexpr uint32_t idesc = idesc_e4m3_f32(128, N);
         const uint32_t q_addr = smem_u32(q_s);
         for (int t = 0; t < ntiles; ++t) {
           const int s = t % STAGES;
           const int a = t % NUM_ACC;
-          if (!mbar_wait(&full[s], (t / STAGES) & 1, budget, abort_flag, p.err)) break;
-          if (!mbar_wait(&acc_empty[a], ((t / NUM_ACC) & 1) ^ 1, budget, abort_flag, p.err)) break;
+          if (!mbar_wait_sleep(&full[s], (t / STAGES) & 1, budget, abort_flag, p.err)) break;
+          if (!mbar_wait_sleep(&acc_empty[a], ((t / NUM_ACC) & 1) ^ 1, budget, abort_flag, p.err)) break;
           tc_fence_after();
           const uint32_t k_addr = smem_u32(k_s + s * kTileBytes);
           const uint32_t d = tmem_base + static_cast<uint32_t>(a * N);
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
     bool w_ok = true;
     if (ntiles > 0) {
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(q_full, 0, budget, abort_flag, p.err) ? 1 : 0;
+      if (lane == 0) ok = mbar_wait_sleep(q_full, 0, budget, abort_flag, p.err) ? 1 : 0;
       w_ok = __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
     }
     if constexpr (W_REGS) {
@@ -327,9 +327,9 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
       int ok = 1;
       if (lane == 0) {
         if constexpr (C::kOneCommit)   // the stage's release commit also marks the tile's MMAs done
-          ok = mbar_wait(&empty[t % STAGES], (t / STAGES) & 1, budget, abort_flag, p.err) ? 1 : 0;
+          ok = mbar_wait_sleep(&empty[t % STAGES], (t / STAGES) & 1, budget, abort_flag, p.err) ? 1 : 0;
         else
-          ok = mbar_wait(&acc_full[a], (t / NUM_ACC) & 1, budget, abort_flag, p.err) ? 1 : 0;
+          ok = mbar_wait_sleep(&acc_full[a], (t / NUM_ACC) & 1, budget, abort_flag, p.err) ? 1 : 0;
       }
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
