@@ -1052,11 +1052,16 @@ __device__ __forceinline__ uint32_t fine_suffix_above(const uint32_t* hist, int 
 
 // Returns true when out[0 … kt) holds the positions of the kt best of keys[0 … vis)
 // (0 < kt < vis ≤ 65536: positions are listed as 16-bit; keys 16-byte aligned).
+// tr: per-CTA phase stamps (slots 8-11: range, bounds, pass, each level), or null.
 template <typename K>
 __device__ bool sampled_select_row(const K* keys, int vis, int kt, uint16_t* list_a, int cap_a, uint16_t* list_b,
-                                   int cap_b, uint32_t* hist, int32_t* out, SampledSmem<K>& ss) {
+                                   int cap_b, uint32_t* hist, int32_t* out, SampledSmem<K>& ss,
+                                   unsigned long long* tr = nullptr) {
   using O = KeyOps<K>;
   const int tid = threadIdx.x, nthr = blockDim.x, warp = tid >> 5, lane = tid & 31;
+  auto stamp = [&](int slot) {
+    if (tr && tid == 0) tr[slot] = globaltimer_ns();
+  };
   const int S = vis < kSampleMax ? vis : kSampleMax;
   // ---- the sample's range
   K lo = O::highest(), hi = O::lowest();
@@ -1066,6 +1071,7 @@ __device__ bool sampled_select_row(const K* keys, int vis, int kt, uint16_t* lis
     hi = O::hi(hi, v);
   }
   block_min_max(lo, hi, ss);
+  stamp(8);
   const float scale = static_cast<float>(kFineBins) / O::diff(hi, lo);
   if (!(hi > lo) || !O::finite(lo) || !O::finite(hi) || !isfinite(scale)) return false;
   for (int b = tid; b < kFineBins; b += nthr) hist[b] = 0u;
@@ -1103,6 +1109,7 @@ __device__ bool sampled_select_row(const K* keys, int vis, int kt, uint16_t* lis
     }
   }
   __syncthreads();
+  stamp(9);
   const K t_hi = ss.t_hi, t_lo = ss.t_lo;
   // ---- one pass: certain members out, candidates listed
   const uint32_t lt = lanemask_lt();
@@ -1150,6 +1157,7 @@ __device__ bool sampled_select_row(const K* keys, int vis, int kt, uint16_t* lis
     }
   }
   __syncthreads();
+  stamp(10);
   const int n_in = ss.cnt_in;
   int m = ss.cnt_set;
   if (n_in > kt || n_in + m < kt || m > cap_a) return false;
@@ -1223,6 +1231,7 @@ __device__ bool sampled_select_row(const K* keys, int vis, int kt, uint16_t* lis
     filled += take;
     need -= take;
     m = ss.cnt_next;
+    stamp(11);
     uint16_t* t = set;
     set = next;
     next = t;

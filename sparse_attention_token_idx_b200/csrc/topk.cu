@@ -245,9 +245,10 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(const RowParam
     // (bound from the first chunk, list, levels) when one of its checks fails
     bool landed = true;
     for (int c = 0; c < nchunks && landed; ++c) landed = wait_chunk(c);
+    if (tr && tid == 0) tr[1] = globaltimer_ns();
     if (landed) {
       if (sampled_select_row<float>(reinterpret_cast<const float*>(keys), vis, kt, list16, p.list_cap, cand16,
-                                    p.cand_cap, hist1, out, ss)) {
+                                    p.cand_cap, hist1, out, ss, tr)) {
         for (int t = kt + tid; t < p.k; t += nthr) out[t] = -1;
         if (tr && tid == 0) tr[4] = globaltimer_ns();
         return;
