@@ -916,330 +916,4 @@ __device__ __forceinline__ void cluster_select_row(SelectSmem& sm, const uint32_
   }
 }
 
-// ---------------------------------------------------------------------------
-// Sampled selection of one row held in shared memory (floats, or order keys
-// as uint32 — both compare as the scores do, floats with −0 equal to +0).
-// A strided sample of S keys, binned linearly between its least and greatest
-// value, estimates where the kt-th best lies; bounds a few standard deviations
-// of the sample count either side of it split the row, in one pass, into keys
-// certainly in (≥ T_hi: written out directly), candidates (T_lo ≤ v < T_hi:
-// listed) and the rest.  The candidates are then narrowed by linear bins over
-// their own range until the rest tie or all are taken.  Every step is checked
-// (in-count ≤ kt ≤ in-count + candidates, lists within capacity, finite
-// ranges, at most kRefineLevels levels); when a check fails the function
-// returns false and the caller runs the exact radix selection, which rewrites
-// every output slot.
-
-constexpr int kSampleLog = 12;
-constexpr int kSampleMax = 1 << kSampleLog;   // sample size for rows of at least that many keys
-
-// Position of sample j of a row of vis keys: every key of a short row, else
-// ⌊j · vis / 4096⌋ (j · vis < 2^28 for rows of up to 65 536 keys).
-__device__ __forceinline__ int sample_pos(int j, int vis) {
-  return vis < kSampleMax ? j : (j * vis) >> kSampleLog;
-}
-constexpr int kFineBins = 1024;
-constexpr int kRefineLevels = 8;
-
-template <typename K>
-struct KeyOps;
-
-template <>
-struct KeyOps<float> {
-  static __device__ __forceinline__ float lowest() { return -INFINITY; }
-  static __device__ __forceinline__ float highest() { return INFINITY; }
-  static __device__ __forceinline__ float lo(float a, float b) { return fminf(a, b); }
-  static __device__ __forceinline__ float hi(float a, float b) { return fmaxf(a, b); }
-  static __device__ __forceinline__ float diff(float v, float mn) { return v - mn; }
-  static __device__ __forceinline__ float edge(float mn, int b, float scale) { return mn + static_cast<float>(b) / scale; }
-  static __device__ __forceinline__ float above(float v) {   // the next value above v
-    return __int_as_float(__float_as_int(v) + (v >= 0.f ? 1 : -1));
-  }
-  static __device__ __forceinline__ bool finite(float v) { return isfinite(v); }
-  static __device__ __forceinline__ float shfl_xor(float v, int o) { return __shfl_xor_sync(0xFFFFFFFFu, v, o); }
-  static __device__ __forceinline__ float from_bits(uint32_t u) { return __uint_as_float(u); }
-};
-
-// Order keys (order_key of the scores): compared as integers, binned by the
-// scores they encode, so that bins are linear in the score as for floats.
-template <>
-struct KeyOps<uint32_t> {
-  static __device__ __forceinline__ float value(uint32_t u) {
-    return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
-  }
-  static __device__ __forceinline__ uint32_t lowest() { return 0u; }
-  static __device__ __forceinline__ uint32_t highest() { return 0xFFFFFFFFu; }
-  static __device__ __forceinline__ uint32_t lo(uint32_t a, uint32_t b) { return min(a, b); }
-  static __device__ __forceinline__ uint32_t hi(uint32_t a, uint32_t b) { return max(a, b); }
-  static __device__ __forceinline__ float diff(uint32_t v, uint32_t mn) { return value(v) - value(mn); }
-  static __device__ __forceinline__ uint32_t edge(uint32_t mn, int b, float scale) {
-    return order_key(value(mn) + static_cast<float>(b) / scale);
-  }
-  static __device__ __forceinline__ uint32_t above(uint32_t v) { return v == 0xFFFFFFFFu ? v : v + 1u; }
-  static __device__ __forceinline__ bool finite(uint32_t v) { return isfinite(value(v)); }
-  static __device__ __forceinline__ uint32_t shfl_xor(uint32_t v, int o) { return __shfl_xor_sync(0xFFFFFFFFu, v, o); }
-  static __device__ __forceinline__ uint32_t from_bits(uint32_t u) { return u; }
-};
-
-template <typename K>
-struct SampledSmem {
-  K red_lo[32], red_hi[32];
-  K t_lo, t_hi;
-  int cnt_in, cnt_set, cnt_next, b_star, take;
-};
-
-// Block-wide min and max (every thread gets both).
-template <typename K>
-__device__ __forceinline__ void block_min_max(K& lo, K& hi, SampledSmem<K>& ss) {
-  using O = KeyOps<K>;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lo = O::lo(lo, O::shfl_xor(lo, o));
-    hi = O::hi(hi, O::shfl_xor(hi, o));
-  }
-  if (lane == 0) {
-    ss.red_lo[warp] = lo;
-    ss.red_hi[warp] = hi;
-  }
-  __syncthreads();
-  lo = lane < nw ? ss.red_lo[lane] : O::highest();
-  hi = lane < nw ? ss.red_hi[lane] : O::lowest();
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lo = O::lo(lo, O::shfl_xor(lo, o));
-    hi = O::hi(hi, O::shfl_xor(hi, o));
-  }
-  __syncthreads();   // the reduction slots may be reused right after
-}
-
-template <typename K>
-__device__ __forceinline__ int fine_bin(K v, K mn, float scale) {
-  return static_cast<int>(fminf(KeyOps<K>::diff(v, mn) * scale, static_cast<float>(kFineBins - 1)));
-}
-
-// Warp-aggregated append of the lanes with `pred` to dst[*counter …]; entries at
-// or past cap are counted but not stored.  All lanes of the warp call it.
-template <typename T>
-__device__ __forceinline__ void warp_append(bool pred, T value, int* counter, T* dst, int cap) {
-  const uint32_t m = __ballot_sync(0xFFFFFFFFu, pred);
-  if (m == 0u) return;
-  const int lane = threadIdx.x & 31;
-  const int leader = __ffs(m) - 1;
-  int base = 0;
-  if (lane == leader) base = atomicAdd(counter, __popc(m));
-  base = __shfl_sync(0xFFFFFFFFu, base, leader);
-  const int q = base + __popc(m & lanemask_lt());
-  if (pred && q < cap) dst[q] = value;
-}
-
-// Warp 0: C(b) = entries in bins ≥ b of hist[0 … kFineBins); returns, in every
-// lane, the suffix count above this lane's 32 bins (the lane's own bins are
-// walked by the caller from the top).
-__device__ __forceinline__ uint32_t fine_suffix_above(const uint32_t* hist, int lane) {
-  constexpr int per = kFineBins / 32;
-  uint32_t own = 0;
-#pragma unroll 8
-  for (int q = 0; q < per; ++q) own += hist[lane * per + q];
-  uint32_t above = own;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_down_sync(0xFFFFFFFFu, above, o);
-    if (lane + o < 32) above += t;
-  }
-  return above - own;
-}
-
-// Returns true when out[0 … kt) holds the positions of the kt best of keys[0 … vis)
-// (0 < kt < vis ≤ 65536: positions are listed as 16-bit; keys 16-byte aligned).
-// tr: per-CTA phase stamps (slots 8-11: range, bounds, pass, each level), or null.
-template <typename K>
-__device__ bool sampled_select_row(const K* keys, int vis, int kt, uint16_t* list_a, int cap_a, uint16_t* list_b,
-                                   int cap_b, uint32_t* hist, int32_t* out, SampledSmem<K>& ss,
-                                   unsigned long long* tr = nullptr) {
-  using O = KeyOps<K>;
-  const int tid = threadIdx.x, nthr = blockDim.x, warp = tid >> 5, lane = tid & 31;
-  auto stamp = [&](int slot) {
-    if (tr && tid == 0) tr[slot] = globaltimer_ns();
-  };
-  const int S = vis < kSampleMax ? vis : kSampleMax;
-  // ---- the sample's range
-  K lo = O::highest(), hi = O::lowest();
-  for (int j = tid; j < S; j += nthr) {
-    const K v = keys[sample_pos(j, vis)];
-    lo = O::lo(lo, v);
-    hi = O::hi(hi, v);
-  }
-  block_min_max(lo, hi, ss);
-  stamp(8);
-  const float scale = static_cast<float>(kFineBins) / O::diff(hi, lo);
-  if (!(hi > lo) || !O::finite(lo) || !O::finite(hi) || !isfinite(scale)) return false;
-  for (int b = tid; b < kFineBins; b += nthr) hist[b] = 0u;
-  if (tid == 0) {
-    ss.cnt_in = 0;
-    ss.cnt_set = 0;
-  }
-  __syncthreads();
-  for (int j = tid; j < S; j += nthr)
-    atomicAdd(&hist[fine_bin(keys[sample_pos(j, vis)], lo, scale)], 1u);
-  __syncthreads();
-  // ---- bounds: T_hi where C(b) drops to r − δ, T_lo where it reaches r + δ
-  if (warp == 0) {
-    constexpr int per = kFineBins / 32;
-    const float p = static_cast<float>(kt) / static_cast<float>(vis);
-    const float r = p * static_cast<float>(S);
-    const float delta = 4.0f * sqrtf(static_cast<float>(S) * p * (1.0f - p)) + 2.0f;
-    const float lim_hi = r - delta, lim_lo = r + delta;
-    int b_hi = kFineBins, b_lo = -1;
-    uint32_t c = fine_suffix_above(hist, lane);
-    for (int q = per - 1; q >= 0; --q) {
-      const int b = lane * per + q;
-      c += hist[b];   // C(b)
-      if (static_cast<float>(c) <= lim_hi) b_hi = b;
-      if (static_cast<float>(c) >= lim_lo && b > b_lo) b_lo = b;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      b_hi = min(b_hi, __shfl_xor_sync(0xFFFFFFFFu, b_hi, o));
-      b_lo = max(b_lo, __shfl_xor_sync(0xFFFFFFFFu, b_lo, o));
-    }
-    if (lane == 0) {
-      ss.t_hi = b_hi >= kFineBins ? O::above(hi) : O::edge(lo, b_hi, scale);
-      ss.t_lo = b_lo < 0 ? O::lowest() : O::edge(lo, b_lo, scale);
-    }
-  }
-  __syncthreads();
-  stamp(9);
-  const K t_hi = ss.t_hi, t_lo = ss.t_lo;
-  // ---- one pass: certain members out, candidates listed
-  const uint32_t lt = lanemask_lt();
-  for (int base = 0; base < vis; base += 4 * nthr) {
-    const int i0 = base + 4 * tid;
-    K v4[4];
-    if (i0 + 3 < vis) {   // keys is 16-byte aligned
-      const uint4 w = *reinterpret_cast<const uint4*>(keys + i0);
-      v4[0] = O::from_bits(w.x);
-      v4[1] = O::from_bits(w.y);
-      v4[2] = O::from_bits(w.z);
-      v4[3] = O::from_bits(w.w);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) v4[e] = i0 + e < vis ? keys[i0 + e] : O::lowest();
-    }
-    uint32_t mi[4], mc[4];
-    int ti = 0, tc = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const bool live = i0 + e < vis;
-      const K v = v4[e];
-      const bool in = live && v >= t_hi;
-      const bool cand = live && !in && v >= t_lo;
-      mi[e] = __ballot_sync(0xFFFFFFFFu, in);
-      mc[e] = __ballot_sync(0xFFFFFFFFu, cand);
-      ti += __popc(mi[e]);
-      tc += __popc(mc[e]);
-    }
-    if (ti + tc == 0) continue;
-    int bi = 0, bc = 0;
-    if (lane == 0) {
-      if (ti) bi = atomicAdd(&ss.cnt_in, ti);
-      if (tc) bc = atomicAdd(&ss.cnt_set, tc);
-    }
-    bi = __shfl_sync(0xFFFFFFFFu, bi, 0);
-    bc = __shfl_sync(0xFFFFFFFFu, bc, 0);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int qi = bi + __popc(mi[e] & lt), qc = bc + __popc(mc[e] & lt);
-      if ((mi[e] >> lane & 1u) && qi < kt) out[qi] = i0 + e;
-      if ((mc[e] >> lane & 1u) && qc < cap_a) list_a[qc] = static_cast<uint16_t>(i0 + e);
-      bi += __popc(mi[e]);
-      bc += __popc(mc[e]);
-    }
-  }
-  __syncthreads();
-  stamp(10);
-  const int n_in = ss.cnt_in;
-  int m = ss.cnt_set;
-  if (n_in > kt || n_in + m < kt || m > cap_a) return false;
-  // ---- narrow the candidates: `set` holds m entries, `need` of them are taken
-  int need = kt - n_in, filled = n_in;
-  uint16_t* set = list_a;
-  uint16_t* next = list_b;
-  int cap_set = cap_a, cap_next = cap_b;
-  for (int level = 0; level < kRefineLevels; ++level) {
-    if (need == 0) return true;
-    K mn = O::highest(), mx = O::lowest();
-    for (int j = tid; j < m; j += nthr) {
-      const K x = keys[set[j]];
-      mn = O::lo(mn, x);
-      mx = O::hi(mx, x);
-    }
-    block_min_max(mn, mx, ss);
-    if (need == m || !(mx > mn)) {
-      // all of the set, or `need` of equal values: the first ones in list order
-      for (int j = tid; j < need; j += nthr) out[filled + j] = set[j];
-      return true;
-    }
-    const float sc = static_cast<float>(kFineBins) / O::diff(mx, mn);
-    if (!isfinite(sc)) return false;
-    for (int b = tid; b < kFineBins; b += nthr) hist[b] = 0u;
-    if (tid == 0) {
-      ss.cnt_in = 0;
-      ss.cnt_next = 0;
-    }
-    __syncthreads();
-    for (int j = tid; j < m; j += nthr) atomicAdd(&hist[fine_bin(keys[set[j]], mn, sc)], 1u);
-    __syncthreads();
-    if (warp == 0) {   // b* = the largest bin with C(b*) ≥ need; take = C(b* + 1)
-      constexpr int per = kFineBins / 32;
-      int bs = -1;
-      uint32_t take = 0, c = fine_suffix_above(hist, lane);
-      for (int q = per - 1; q >= 0; --q) {
-        const int b = lane * per + q;
-        const uint32_t c_next = c;
-        c += hist[b];
-        if (c >= static_cast<uint32_t>(need) && c_next < static_cast<uint32_t>(need)) {
-          bs = b;
-          take = c_next;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const int obs = __shfl_xor_sync(0xFFFFFFFFu, bs, o);
-        const uint32_t otk = __shfl_xor_sync(0xFFFFFFFFu, take, o);
-        if (obs > bs) {
-          bs = obs;
-          take = otk;
-        }
-      }
-      if (lane == 0) {
-        ss.b_star = bs;
-        ss.take = static_cast<int>(take);
-      }
-    }
-    __syncthreads();
-    const int bs = ss.b_star, take = ss.take;
-    if (bs < 0 || static_cast<int>(hist[bs]) > cap_next) return false;
-    for (int base = 0; base < m; base += nthr) {
-      const int j = base + tid;
-      const int pos = j < m ? set[j] : 0;
-      const int b = j < m ? fine_bin(keys[pos], mn, sc) : -1;
-      warp_append<int32_t>(b > bs, pos, &ss.cnt_in, out + filled, take);
-      warp_append<uint16_t>(b == bs, static_cast<uint16_t>(pos), &ss.cnt_next, next, cap_next);
-    }
-    __syncthreads();
-    filled += take;
-    need -= take;
-    m = ss.cnt_next;
-    stamp(11);
-    uint16_t* t = set;
-    set = next;
-    next = t;
-    const int tc2 = cap_set;
-    cap_set = cap_next;
-    cap_next = tc2;
-  }
-  return need == 0;
-}
-
 }  // namespace idx

@@ -152,7 +152,6 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(const RowParam
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L.keys);   // fp32 scores until converted
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   __shared__ int timed_out;
-  __shared__ SampledSmem<float> ss;
   const int tid = threadIdx.x, nthr = blockDim.x;
   unsigned long long* tr = (p.trace && blockIdx.x < 8192) ? p.trace + blockIdx.x * kTraceSlotsT : nullptr;
   if (tr && tid == 0) tr[0] = globaltimer_ns();
@@ -240,24 +239,6 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(const RowParam
     }
     return !__syncthreads_or(timed_out);
   };
-  if (use_list) {
-    // the sampled selection over the whole row first; the radix path below
-    // (bound from the first chunk, list, levels) when one of its checks fails
-    bool landed = true;
-    for (int c = 0; c < nchunks && landed; ++c) landed = wait_chunk(c);
-    if (tr && tid == 0) tr[1] = globaltimer_ns();
-    if (landed) {
-      if (sampled_select_row<float>(reinterpret_cast<const float*>(keys), vis, kt, list16, p.list_cap, cand16,
-                                    p.cand_cap, hist1, out, ss, tr)) {
-        for (int t = kt + tid; t < p.k; t += nthr) out[t] = -1;
-        if (tr && tid == 0) tr[4] = globaltimer_ns();
-        return;
-      }
-      __syncthreads();
-      for (int t = tid; t < kHistBins; t += nthr) hist1[t] = 0u;
-      __syncthreads();
-    }
-  }
   bool ok = true;
   for (int c = 0; c < nchunks && ok; ++c) {
     ok = wait_chunk(c);

@@ -47,7 +47,7 @@ ROWS = [
     ("large-k", 64, 16384, 16384, 4096, "random"),     # positions written without staging
     ("ragged", 80, 16381, 16384, 512, "random"),       # lengths not multiples of 4 (ld is)
     ("unaligned-ld", 70, 3001, 3001, 700, "random"),   # ld % 4 != 0: cluster kernel
-    ("sample-blind", 64, 16384, 16384, 2048, "strided"),  # the sampled positions all score low: radix fallback
+    ("strided-low", 64, 16384, 16384, 2048, "strided"),   # every 4th position far below the rest
 ]
 
 
@@ -121,13 +121,11 @@ def test_fused_topk_matches_oracle_and_unfused(name, B, n, positions, T_cap, cau
             check_topk_exact_row(idx[b, i], sc[b, i], vis, k)
 
 
-@pytest.mark.parametrize("zeroed", ["all", "sampled-positions"])
-def test_fused_topk_when_the_sample_cannot_place_the_threshold(zeroed):
-    """The one-CTA decode selection first estimates the threshold from a strided
-    sample of the row; when the sample has no spread (every sampled key scores
-    0) it hands the row to the exact radix selection.  Keys zeroed at every
-    position (all scores tie) or only at the sampled positions (every 4th of
-    16 384) must still give an exact top-k."""
+@pytest.mark.parametrize("zeroed", ["all", "every-4th"])
+def test_fused_topk_with_zeroed_keys(zeroed):
+    """The fused decode selection on degenerate score rows: keys zeroed at
+    every position (all scores tie at 0) or at every 4th of 16 384 positions
+    (a quarter of the row ties at 0).  The top-k must still be exact."""
     from sparse_attention_token_idx_b200 import binding as X
     B, T_cap, k = 4, 16384, 2048
     case = synth.make_case("zeroed-" + zeroed, 77, B, 1, [T_cap - 1] * B, T_cap=T_cap, causal=False, fmt=1, k=k)
