@@ -302,16 +302,18 @@ def measure(args, widx, dev, world, headline):
         raise RuntimeError(f"device error in the timed region: status {code}, bits {bits}")
 
     # -------------------------------------------------------------- end to end from pinned host memory
-    h_k = case_pinned(torch, case.k_new.view(np.int16)).view(torch.bfloat16)
-    h_q = case_pinned(torch, case.q.view(np.int16)).view(torch.bfloat16)
-    h_w = case_pinned(torch, case.w_raw)
-    h_p = case_pinned(torch, case.positions)
-    h_l = case_pinned(torch, case.lengths)
-    h_out = torch.empty((B, n, case.k), dtype=torch.int32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (h_k, h_q, h_w, h_p, h_l))
-    d2h = h_out.numel() * h_out.element_size()
-    # uploads, compute and downloads on three streams, two slots of device buffers (HostPipeline)
+    # uploads, compute and downloads on three streams, two slots of device buffers (HostPipeline);
+    # the step's inputs sit in one pinned buffer with the device layout: one upload per step
     hp = HostPipeline(ix, B, n, causal=case.causal, max_len=max_len)
+    h_k, h_q, h_w, h_p, h_l = hp.host_inputs()
+    h_k.copy_(case_pinned(torch, case.k_new.view(np.int16)).view(torch.bfloat16))
+    h_q.copy_(case_pinned(torch, case.q.view(np.int16)).view(torch.bfloat16))
+    h_w.copy_(case_pinned(torch, case.w_raw))
+    h_p.copy_(case_pinned(torch, case.positions))
+    h_l.copy_(case_pinned(torch, case.lengths))
+    h_out = torch.empty((B, n, case.k), dtype=torch.int32).pin_memory()
+    h2d = hp.packed_bytes
+    d2h = h_out.numel() * h_out.element_size()
 
     def step_e2e():
         hp.submit(h_k, h_q, h_w, h_p, h_l, h_out)

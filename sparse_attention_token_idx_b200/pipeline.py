@@ -138,22 +138,46 @@ class HostPipeline:
     the step itself.
     """
 
+    # the step's inputs, in the order they are packed: name, shape (B, n), dtype
+    FIELDS = (("k", lambda B, n: (B, n, X.DIM), torch.bfloat16),
+              ("q", lambda B, n: (B, n, X.HEADS, X.DIM), torch.bfloat16),
+              ("w", lambda B, n: (B, n, X.HEADS), torch.float32),
+              ("p", lambda B, n: (B,), torch.int32),
+              ("l", lambda B, n: (B,), torch.int32))
+
+    def _layout(self):
+        """(name, shape, dtype, byte offset) of each input in a packed buffer
+        (offsets rounded up to 256 bytes), and the buffer's size."""
+        out, off = [], 0
+        for name, shape_of, dt in self.FIELDS:
+            shape = shape_of(self.B, self.n)
+            nbytes = torch.Size(shape).numel() * torch.empty((), dtype=dt).element_size()
+            out.append((name, shape, dt, off))
+            off = (off + nbytes + 255) // 256 * 256
+        return out, off
+
+    def _views(self, buf):
+        return {name: buf[off:off + torch.Size(shape).numel() * torch.empty((), dtype=dt).element_size()]
+                .view(dt).view(shape) for name, shape, dt, off in self.layout}
+
     def __init__(self, indexer: Indexer, B: int, n: int, *, causal: bool, max_len: int, slots: int = 2):
         if slots < 1:
             raise ValueError("slots must be ≥ 1")
         dev = indexer.device
         self.ix, self.causal, self.max_len = indexer, causal, max_len
+        self.B, self.n = B, n
+        self.layout, self.packed_bytes = self._layout()
+        self.packed_hosts = {}      # data_ptr of a host_inputs() buffer → that buffer
         self.up = torch.cuda.Stream(device=dev)
         self.comp = torch.cuda.Stream(device=dev)
         self.down = torch.cuda.Stream(device=dev)
         self.slots = []
         for _ in range(slots):
+            packed = torch.empty((self.packed_bytes,), dtype=torch.uint8, device=dev)
+            v = self._views(packed)
             self.slots.append({
-                "k": torch.empty((B, n, X.DIM), dtype=torch.bfloat16, device=dev),
-                "q": torch.empty((B, n, X.HEADS, X.DIM), dtype=torch.bfloat16, device=dev),
-                "w": torch.empty((B, n, X.HEADS), dtype=torch.float32, device=dev),
-                "p": torch.empty((B,), dtype=torch.int32, device=dev),
-                "l": torch.empty((B,), dtype=torch.int32, device=dev),
+                "packed": packed,
+                "k": v["k"], "q": v["q"], "w": v["w"], "p": v["p"], "l": v["l"],
                 "out": torch.empty((B, n, indexer.k), dtype=torch.int32, device=dev),
                 "graph": None,
                 "uploaded": torch.cuda.Event(),
@@ -174,19 +198,44 @@ class HostPipeline:
         stream.wait_stream(self.comp)
         stream.wait_stream(self.down)
 
+    def host_inputs(self):
+        """Pinned host tensors (k_new, q, w_raw, positions, lengths) packed in one
+        buffer with the device slots' layout: a step submitted with exactly these
+        views is uploaded by a single copy.  Allocate several for rotation."""
+        buf = torch.empty((self.packed_bytes,), dtype=torch.uint8).pin_memory()
+        self.packed_hosts[buf.data_ptr()] = buf
+        v = self._views(buf)
+        return v["k"], v["q"], v["w"], v["p"], v["l"]
+
+    def _packed_of(self, hs):
+        """The host_inputs() buffer that the five tensors are the views of, or None."""
+        buf = self.packed_hosts.get(hs[0].data_ptr())
+        if buf is None:
+            return None
+        base = buf.data_ptr()
+        for h, (name, shape, dt, off) in zip(hs, self.layout):
+            if h.data_ptr() != base + off or tuple(h.shape) != tuple(shape) or h.dtype != dt:
+                return None
+        return buf
+
     def submit(self, h_k, h_q, h_w, h_p, h_l, h_out) -> torch.cuda.Event:
         """One step: pinned host inputs k_new [B, n, 128] bf16, q [B, n, 64, 128]
-        bf16, w_raw [B, n, 64] fp32, positions [B], lengths [B] int32; the
-        indices land in pinned h_out [B, n, k] int32 once the returned event
-        has completed.  Refill the host inputs (or reuse h_out) only after that
-        event, or rotate several host buffers."""
+        bf16, w_raw [B, n, 64] fp32, positions [B], lengths [B] int32 (the views
+        of one host_inputs() buffer: a single upload); the indices land in
+        pinned h_out [B, n, k] int32 once the returned event has completed.
+        Refill the host inputs (or reuse h_out) only after that event, or
+        rotate several host buffers."""
         s = self.slots[self.count % len(self.slots)]
         self.count += 1
         if s["used"]:
             self.up.wait_event(s["computed"])        # the slot's inputs are free once its last step computed
+        packed = self._packed_of((h_k, h_q, h_w, h_p, h_l))
         with torch.cuda.stream(self.up):
-            for name, h in (("k", h_k), ("q", h_q), ("w", h_w), ("p", h_p), ("l", h_l)):
-                s[name].copy_(h, non_blocking=True)
+            if packed is not None:            # one copy for the whole step
+                s["packed"].copy_(packed, non_blocking=True)
+            else:
+                for name, h in (("k", h_k), ("q", h_q), ("w", h_w), ("p", h_p), ("l", h_l)):
+                    s[name].copy_(h, non_blocking=True)
         s["uploaded"].record(self.up)
         self.comp.wait_event(s["uploaded"])
         if s["used"]:

@@ -136,3 +136,39 @@ def test_host_pipeline_matches_eager_steps_in_order():
             newer = set(range(base[b], base[b] + j))                # keys appended by the earlier steps
             assert newer <= set(got[b, 0].tolist()), f"step {j} sequence {b} misses an earlier step's key"
     assert torch.equal(ixs[0].k_cache, ixs[1].k_cache) and torch.equal(ixs[0].k_scale_cache, ixs[1].k_scale_cache)
+
+
+def test_host_pipeline_packed_inputs_match_separate_ones():
+    """The same decode step submitted from host_inputs() views (one upload)
+    and from separate pinned tensors (five uploads) selects the same sets."""
+    from sparse_attention_token_idx_b200 import binding as X
+    from sparse_attention_token_idx_b200.pipeline import HostPipeline, Indexer
+    B, k = 3, 64
+    case = synth.make_case("hp-packed", 530, B, 1, [700, 1500, 90], T_cap=2048, k=k, fmt=0)
+    outs = []
+    for packed in (False, True):
+        ix = Indexer(B, case.T_cap, case.fmt, k)
+        for b in range(B):
+            p = int(case.positions[b])
+            X.quant_append(bf16_dev(case.k_prior[b:b + 1, :p]), dev(np.zeros(1, np.int32)), ix.k_cache[b:b + 1],
+                           ix.k_scale_cache[b:b + 1], case.fmt)
+        hp = HostPipeline(ix, B, 1, causal=False, max_len=int(case.lengths.max()))
+        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+        srcs = (pin(case.k_new.view(np.int16)).view(torch.bfloat16), pin(case.q.view(np.int16)).view(torch.bfloat16),
+                pin(case.w_raw), pin(case.positions), pin(case.lengths))
+        if packed:
+            hs = hp.host_inputs()
+            for h, src in zip(hs, srcs):
+                h.copy_(src)
+            assert hp._packed_of(hs) is not None
+        else:
+            hs = srcs
+            assert hp._packed_of(hs) is None
+        h_out = torch.empty((B, 1, k), dtype=torch.int32).pin_memory()
+        hp.submit(*hs, h_out)
+        hp.join()
+        torch.cuda.synchronize()
+        assert X.status() == (0, 0)
+        outs.append(h_out.numpy().copy())
+    for b in range(B):
+        assert set(outs[0][b, 0].tolist()) == set(outs[1][b, 0].tolist())
