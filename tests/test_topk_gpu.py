@@ -91,6 +91,9 @@ FUSED = [
     # 64 decode rows, fewer than the SMs: the fused kernel splits each row over
     # a cluster of 2 CTAs that select through distributed shared memory
     ("decode-many", 64, 1, list(range(1000, 2024, 16)), 2048, False, 1, 256),
+    # more than half as many rows as SMs: one CTA per row, ragged lengths
+    ("decode-100", 100, 1, [1000 + 31 * i for i in range(100)], 4096, False, 0, 256),
+    ("decode-n2", 60, 2, [500 + 60 * i for i in range(60)], 4096, True, 1, 128),
 ]
 
 
