@@ -114,7 +114,11 @@ struct Cfg {
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT, bool W_REGS>
+// CL: a fused call whose rows are split over a cluster (G > 1).  Fused calls
+// with one CTA per row use the CL = false instance, which carries only the
+// one-CTA selection: a smaller kernel, whose selection code stays in the
+// instruction cache from one launch to the next.
+template <int NT, bool FUSED, int STAGES, int NUM_ACC, int EPI_WARPS, int TSPLIT, bool W_REGS, bool CL>
 __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>::kThreads,
                                   Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>::kMinCtas)
     score_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
@@ -157,8 +161,8 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
   }
   // fused calls split a row over a cluster (the selection exchanges through
   // distributed shared memory); unfused calls split it over plain CTAs
-  const uint32_t rank = FUSED ? cluster_rank() : static_cast<uint32_t>(blockIdx.x % p.G);
-  const int G = p.G;
+  const uint32_t rank = FUSED ? (CL ? cluster_rank() : 0u) : static_cast<uint32_t>(blockIdx.x % p.G);
+  const int G = (FUSED && !CL) ? 1 : p.G;
   const int item = blockIdx.x / G;
   const int b = item % p.B;
   const int tb = p.ntb - 1 - item / p.B;   // longest (latest) row blocks first
@@ -437,7 +441,7 @@ __global__ void __launch_bounds__(Cfg<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSP
           for (int i = kt + threadIdx.x; i < p.k; i += blockDim.x) out[i] = -1;
       }
     }
-    if (G > 1) cluster_sync(); else __syncthreads();
+    if (CL && G > 1) cluster_sync(); else __syncthreads();
   }
 
   if (trace && threadIdx.x == 0) tr[4] = globaltimer_ns();
@@ -526,7 +530,9 @@ int launch_score(const uint8_t* q_fp8, const float* w, const uint8_t* k_cache, c
                         kTileKeys))
     return IDX_ERR_ALIGN;
 
-  auto kern = score_kernel<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS>;
+  auto kern = score_kernel<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS, false>;
+  if constexpr (FUSED)
+    if (G > 1) kern = score_kernel<NT, FUSED, STAGES, NUM_ACC, EPI_WARPS, TSPLIT, W_REGS, true>;
   if (const int r = ensure_smem_limit(reinterpret_cast<const void*>(kern), smem)) return r;
   ScoreParams p;
   p.w = w;
