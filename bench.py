@@ -48,6 +48,10 @@ KEY_BYTES = 128 + 4           # one cached key: 128 e4m3 codes + fp32 scale
 ROW_BYTES_IN = 64 * 128 + 64 * 4   # one query row: 64 heads of e4m3 codes + 64 fp32 weights
 PROFILE_SCORE = os.path.join(ROOT, "profiles", "score_topk_decode_b128_t16384.md")
 KERNEL_SOURCES = ["score.cu", "select.cuh", "ptx.cuh"]
+# the prefill scorer's capture (workload 3, one launch) and the sources it was taken from
+PROFILE_FLAT = os.path.join(ROOT, "profiles", "flat_score_prefill_b1_s4096.md")
+FLAT_SOURCES = ["flat_score.cu", "epilogue.cuh", "ptx.cuh"]
+FLAT_PROFILE_WORKLOAD = 3
 
 
 def env_rank():
@@ -63,27 +67,46 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(files=None):
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in files or KERNEL_SOURCES:
         h.update(open(os.path.join(ROOT, "sparse_attention_token_idx_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def profile_traffic(path, launch_units):
-    """DRAM bytes per launch from a committed ncu summary, scaled to this launch's
-    units, or None when the summary is missing or the kernel source changed."""
+def profile_values(path, files):
+    """The `- key: value` lines of a committed ncu summary, or None when it is
+    missing or its source_sha256 no longer matches the kernel's sources."""
     try:
         kv = {}
         for line in open(path):
             if ":" in line and line.strip().startswith("- "):
                 k, v = line.strip()[2:].split(":", 1)
                 kv[k.strip()] = v.strip().strip("`")
-        if kv.get("source_sha256") != kernel_source_hash():
-            return None
-        per_unit = float(kv["dram_bytes_per_key"])
-        return per_unit * launch_units
+        return kv if kv.get("source_sha256") == kernel_source_hash(files) else None
     except Exception:
+        return None
+
+
+def profile_traffic(path, launch_units):
+    """DRAM bytes per launch from a committed ncu summary, scaled to this launch's
+    units, or None when the summary is missing or the kernel source changed."""
+    kv = profile_values(path, KERNEL_SOURCES)
+    try:
+        return float(kv["dram_bytes_per_key"]) * launch_units if kv else None
+    except (KeyError, ValueError):
+        return None
+
+
+def flat_profile_traffic(widx):
+    """DRAM bytes of one prefill-scorer launch, from the committed capture of the
+    workload it was taken on (None for other workloads or a changed source)."""
+    if widx != FLAT_PROFILE_WORKLOAD:
+        return None
+    kv = profile_values(PROFILE_FLAT, FLAT_SOURCES)
+    try:
+        return float(kv["dram_bytes_per_launch"]) if kv else None
+    except (KeyError, ValueError):
         return None
 
 
@@ -345,7 +368,7 @@ def measure(args, widx, dev, world, headline):
     topk_bytes = B * n * 4 * (max_len + case.k) if ws_bytes else None   # score rows read, indices written
     launches_per_step = (3 if (ws_bytes or e8m0) else 2)
     del graph, hp, ix, ws
-    return dict(case=case, e8m0=e8m0, keys=keys, flops=flops, key_rows=key_rows, score_bytes=score_bytes, ms=ms,
+    return dict(widx=widx, case=case, e8m0=e8m0, keys=keys, flops=flops, key_rows=key_rows, score_bytes=score_bytes, ms=ms,
                 score_ms=score_ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
                 clocks=sampler.summary(), launches=launches_per_step * args.steps, topk_ms=topk_ms,
                 topk_bytes=topk_bytes, two_pass=bool(ws_bytes), l2_flushed=flush is not None, n_k=n_k,
@@ -631,7 +654,8 @@ def result_line(r, args, world, hbm, bf16, peak_src):
         achieved = r["flops"] / score_s / 1e12
         peak = bf16 * FP8_PER_BF16
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": None, "peak_source": f"{peak_src} bf16 burst x nominal fp8/bf16 ratio {FP8_PER_BF16}",
+                "traffic": flat_profile_traffic(r["widx"]) if r["two_pass"] and not r["e8m0"] else None,
+                "peak_source": f"{peak_src} bf16 burst x nominal fp8/bf16 ratio {FP8_PER_BF16}",
                 "frac_of_datasheet_fp8": achieved / DATASHEET_FP8_TFLOPS,
                 "kernel": "flat_score_kernel (tcgen05 FP8 scorer, fp32 scores to the workspace)",
                 "kernel_us": r["score_ms"] * 1e3, "algorithmic_flops": r["flops"],
