@@ -368,8 +368,8 @@ def measure(args, widx, dev, world, headline):
     topk_bytes = B * n * 4 * (max_len + case.k) if ws_bytes else None   # score rows read, indices written
     launches_per_step = (3 if (ws_bytes or e8m0) else 2)
     del graph, hp, ix, ws
-    return dict(widx=widx, case=case, e8m0=e8m0, keys=keys, flops=flops, key_rows=key_rows, score_bytes=score_bytes, ms=ms,
-                score_ms=score_ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
+    return dict(widx=widx, case=case, e8m0=e8m0, keys=keys, flops=flops, key_rows=key_rows, score_bytes=score_bytes,
+                ms=ms, score_ms=score_ms, e2e_ms=e2e_ms, e2e_steps=e2e_steps, h2d=h2d, d2h=d2h,
                 clocks=sampler.summary(), launches=launches_per_step * args.steps, topk_ms=topk_ms,
                 topk_bytes=topk_bytes, two_pass=bool(ws_bytes), l2_flushed=flush is not None, n_k=n_k,
                 kernel_clocks=kernel_sampler.summary())
